@@ -1,0 +1,126 @@
+/*
+ * rsa.h -- C ABI of the Ring Self-Attention (RSA) library for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes. "Sequence Parallelism: Making 4D Parallelism Possible" (Li, Xue
+ * et al., 2021; review page, Abstract and "Proposed method") splits a sequence of length L into
+ * N chunks and computes self-attention by passing attention embeddings around a ring of
+ * devices (Ring Self-Attention). The pages give no formula; this library computes exact
+ * softmax attention on the ring schedule, per (batch b, head h):
+ *
+ *   chunk n holds query rows [n*c, (n+1)*c), c = L/N;
+ *   ring pass 1:  S_n[:, block m] = Q_n K_m^T / sqrt(d),  m = (n + s) mod N,  s = 0..N-1
+ *   row softmax over the whole key length: P = exp(S - m_i) / l_i,  lse_i = m_i + ln l_i
+ *   ring pass 2:  O_n = sum_s P_n[:, block m] V_m
+ *
+ * and the backward pass (dQ, dK, dV) on the same schedule. On one GPU the ring's ranks are
+ * chunks resident in one HBM and a ring step is an order of tiles inside the kernels; the
+ * result does not depend on N beyond floating-point rounding.
+ *
+ * Conventions shared by every call:
+ *   - Tensors Q, K, V, O, dO, dQ, dK, dV are contiguous [B, H, L, d] (d fastest) in device
+ *     memory, in the element type `dt` (RSA_BF16: bfloat16; RSA_F32: float). lse is fp32
+ *     [B, H, L]. Base pointers must be 16-byte aligned.
+ *   - scale = 1/sqrt(d) is fixed. causal != 0 keeps keys j <= i only (the diagonal is kept).
+ *     No dropout, bias or padding mask.
+ *   - Supported: B, H, L >= 1, N >= 1 with L % N == 0; bf16 with d in {64, 128}; fp32 with
+ *     d in {32, 64}. L need not be a multiple of any tile size.
+ *   - Arithmetic: bf16 inputs with fp32 accumulation and fp32 softmax statistics; P and dS
+ *     are rounded to bf16 before their GEMMs; outputs are rounded to nearest-even into `dt`.
+ *     The fp32 path computes every step in fp32 on the CUDA cores (no TF32).
+ *   - Ownership: the caller owns every buffer, including `workspace`. The library never
+ *     allocates or frees device memory and never synchronises `stream` (a cudaStream_t;
+ *     NULL means the legacy default stream). Work is enqueued on `stream` in order.
+ *   - Errors: arguments are checked before anything is launched; a failed check returns an
+ *     error code and enqueues nothing. Nothing throws across this interface.
+ */
+#ifndef RSA_H_
+#define RSA_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RSA_API __attribute__((visibility("default")))
+#else
+#define RSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RSA_OK = 0,
+    RSA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, L % N != 0 */
+    RSA_ERR_UNSUPPORTED = 2, /* head dim or dtype outside the supported set, no sm_100 GPU */
+    RSA_ERR_WORKSPACE = 3,   /* workspace smaller than the minimum plan needs */
+    RSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    RSA_ERR_TIMEOUT = 5      /* a kernel's bounded wait ran out (reported afterwards) */
+} rsa_status_t;
+
+typedef enum { RSA_F32 = 0, RSA_BF16 = 1 } rsa_dtype_t;
+
+/*
+ * Bytes of device workspace a call needs.
+ *
+ * The score slab (the c x L block of scores of every chunk, i.e. L x L per head) is
+ * processed in groups: a group is a set of whole heads, or, when one head does not fit, a
+ * range of rows (a multiple of 128) of one head. `budget_bytes` caps the workspace: the
+ * returned size is that of the largest plan that fits the budget (or of the smallest plan if
+ * none fits). budget_bytes == 0 asks for the default plan (at most 1 GiB).
+ * for_backward selects the backward call's needs (it also keeps per-row D_i and, for
+ * row-range groups, fp32 dK/dV accumulators).
+ * Returns 0 if the arguments are invalid or unsupported.
+ */
+RSA_API size_t rsa_workspace_size(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                          int for_backward, size_t budget_bytes);
+
+/*
+ * Forward pass (ring pass 1, row softmax, ring pass 2).
+ * In:  Q, K, V  [B,H,L,d] device, dtype dt.
+ * Out: O [B,H,L,d] device, dtype dt; lse [B,H,L] fp32 device (the softmax statistics the
+ *      backward pass needs; must not be NULL).
+ * workspace: device, >= rsa_workspace_size(..., for_backward = 0, ...) for the plan wanted;
+ *      the plan is the largest one that fits ws_bytes. 256-byte aligned.
+ */
+RSA_API rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, float *lse,
+                         int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Backward pass on the same ring schedule: recomputes P from Q, K and lse, forms
+ * dP = dO V^T and dS = P * (dP - D) with D_i = dO_i . O_i, then
+ * dV_m = sum_n P_n[:, block m]^T dO_n, dK_m = scale sum_n dS_n[:, block m]^T Q_n and
+ * dQ_n = scale sum_s dS_n[:, block m] K_m.
+ * In:  Q, K, V, O, dO [B,H,L,d] device dtype dt; lse [B,H,L] fp32 from rsa_forward.
+ * Out: dQ, dK, dV [B,H,L,d] device dtype dt.
+ * workspace: device, >= rsa_workspace_size(..., for_backward = 1, ...), 256-byte aligned.
+ */
+RSA_API rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const void *O,
+                          const void *dO, const float *lse, void *dQ, void *dK, void *dV,
+                          int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                          void *workspace, size_t ws_bytes, void *stream);
+
+/* Human-readable name of a status code (static string). */
+RSA_API const char *rsa_status_string(rsa_status_t status);
+
+/*
+ * Status reported by kernels since the last call of this function on the current device:
+ * RSA_OK, or RSA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (that kernel then
+ * returned early and its outputs are invalid). Synchronises `stream` and clears the status.
+ */
+RSA_API rsa_status_t rsa_last_device_status(void *stream);
+
+/*
+ * The plan a call with these arguments and ws_bytes would use, for inspection:
+ * out[0] = number of groups, out[1] = heads per group, out[2] = rows per group,
+ * out[3] = padded row length of the slab (elements), out[4] = bytes the plan uses.
+ * Returns RSA_ERR_WORKSPACE if ws_bytes is below the minimum plan.
+ */
+RSA_API rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                               int for_backward, size_t ws_bytes, long long out[5]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSA_H_ */

@@ -1,0 +1,432 @@
+// rsa_abi.cu -- C ABI of the Ring Self-Attention library: argument checks, the slab-group
+// planner, TMA descriptor set-up and the per-group kernel schedule.
+//
+// Ring Self-Attention ("Sequence Parallelism: Making 4D Parallelism Possible", review page,
+// Abstract and "Proposed method") cuts the sequence into N chunks and lets each chunk see
+// every key chunk in ring order. Here all chunks live in one GPU's HBM; the score slabs of
+// the chunks (c x L each, L x L per head) are produced, normalised and consumed group by
+// group so that the workspace stays within a budget. A group is a set of whole heads, or a
+// range of rows (a multiple of 128) of one head when a whole head does not fit.
+#include <cudaTypedefs.h>
+
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "../../include/rsa.h"
+#include "rsa_internal.h"
+
+namespace rsa {
+__device__ int g_status_word;  // RSA_OK or RSA_ERR_TIMEOUT, set by kernels
+}
+
+namespace {
+
+using rsa::Group;
+using rsa::SlabArgs;
+
+constexpr size_t kAlign = 256;
+constexpr size_t kDefaultBudget = size_t(1) << 30;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+    int B, H, L, d, N, causal, bwd;
+    rsa_dtype_t dt;
+    long long BH;
+    int Lp, c;
+    int whole;     // groups of whole heads
+    long long Gh;  // heads per group (whole mode)
+    int R;         // rows per group (row mode); L in whole mode
+    long long ngroups;
+    size_t row_bytes;   // slab bytes per row (all slabs of the pass)
+    size_t slab_bytes;  // slab region
+    size_t off_D, off_acc, total;
+};
+
+bool args_ok(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *why) {
+    if (B <= 0 || H <= 0 || L <= 0 || N <= 0 || d <= 0 || L % N != 0) {
+        *why = RSA_ERR_INVALID_ARG;
+        return false;
+    }
+    if (L > (1 << 22) || static_cast<long long>(B) * H > 0x7fffffffLL) {
+        *why = RSA_ERR_UNSUPPORTED;
+        return false;
+    }
+    if (dt == RSA_BF16) {
+        if (d != 64 && d != 128) {
+            *why = RSA_ERR_UNSUPPORTED;
+            return false;
+        }
+    } else if (dt == RSA_F32) {
+        if (d != 32 && d != 64) {
+            *why = RSA_ERR_UNSUPPORTED;
+            return false;
+        }
+    } else {
+        *why = RSA_ERR_UNSUPPORTED;
+        return false;
+    }
+    return true;
+}
+
+// Largest plan whose workspace fits `budget` (the smallest plan if none does).
+Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, int bwd,
+               size_t budget) {
+    Plan p{};
+    p.B = B, p.H = H, p.L = L, p.d = d, p.N = N, p.causal = causal ? 1 : 0, p.bwd = bwd ? 1 : 0;
+    p.dt = dt;
+    p.BH = static_cast<long long>(B) * H;
+    p.Lp = (L + 63) / 64 * 64;
+    p.c = L / N;
+    // forward: fp32 scores with P written in place; backward: P and dS (bf16, or fp32)
+    p.row_bytes = (dt == RSA_F32 && bwd) ? size_t(8) * p.Lp : size_t(4) * p.Lp;
+    const size_t fixed = bwd ? align_up(size_t(p.BH) * L * 4, kAlign) : 0;
+    const size_t head_bytes = align_up(size_t(L) * p.row_bytes, kAlign);
+    const size_t acc_bytes = (bwd && dt == RSA_BF16) ? 2 * align_up(size_t(L) * d * 4, kAlign) : 0;
+    if (budget >= fixed + head_bytes) {
+        p.whole = 1;
+        long long gh = static_cast<long long>((budget - fixed) / head_bytes);
+        p.Gh = gh < p.BH ? gh : p.BH;
+        p.R = L;
+        p.ngroups = (p.BH + p.Gh - 1) / p.Gh;
+        p.slab_bytes = align_up(size_t(p.Gh) * L * p.row_bytes, kAlign);
+        p.off_D = p.slab_bytes;
+        p.off_acc = p.off_D + fixed;
+        p.total = p.off_acc;
+    } else {
+        p.whole = 0;
+        p.Gh = 1;
+        size_t avail = budget > fixed + acc_bytes ? budget - fixed - acc_bytes : 0;
+        long long r = static_cast<long long>(avail / p.row_bytes) / 128 * 128;
+        if (r < 128) r = 128;
+        if (r >= L) r = L;  // only when L <= 128: a whole head is the minimum plan
+        if (r == L) {
+            p.whole = 1;
+            p.R = L;
+            p.ngroups = p.BH;
+            p.slab_bytes = head_bytes;
+            p.off_D = p.slab_bytes;
+            p.off_acc = p.off_D + fixed;
+            p.total = p.off_acc;
+            return p;
+        }
+        p.R = static_cast<int>(r);
+        const long long per_head = (L + p.R - 1) / p.R;
+        p.ngroups = p.BH * per_head;
+        p.slab_bytes = align_up(size_t(p.R) * p.row_bytes, kAlign);
+        p.off_D = p.slab_bytes;
+        p.off_acc = p.off_D + fixed;
+        p.total = p.off_acc + acc_bytes;
+    }
+    return p;
+}
+
+Group group_of(const Plan &p, long long g) {
+    Group G{};
+    if (p.whole) {
+        G.bh0 = static_cast<int>(g * p.Gh);
+        long long nh = p.BH - g * p.Gh;
+        G.nh = static_cast<int>(nh < p.Gh ? nh : p.Gh);
+        G.r0 = 0;
+        G.R = p.L;
+        G.first_of_head = G.last_of_head = 1;
+    } else {
+        const long long per_head = (p.L + p.R - 1) / p.R;
+        G.bh0 = static_cast<int>(g / per_head);
+        G.nh = 1;
+        const int k = static_cast<int>(g - static_cast<long long>(G.bh0) * per_head);
+        G.r0 = k * p.R;
+        G.R = p.L - G.r0 < p.R ? p.L - G.r0 : p.R;
+        G.first_of_head = k == 0;
+        G.last_of_head = G.r0 + G.R == p.L;
+    }
+    return G;
+}
+
+// ---------------------------------------------------------------- per-device state
+
+struct DeviceState {
+    bool ready;
+    int sms;
+    int *status;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+rsa_status_t device_state(DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return RSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &s = g_dev[dev];
+    if (!s.ready) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return RSA_ERR_CUDA;
+        if (major != 10) return RSA_ERR_UNSUPPORTED;
+        if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return RSA_ERR_CUDA;
+        if (rsa::tc_kernels_configure() != cudaSuccess) return RSA_ERR_CUDA;
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, rsa::g_status_word) != cudaSuccess) return RSA_ERR_CUDA;
+        s.status = static_cast<int *>(ptr);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || !fn)
+                return RSA_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        s.ready = true;
+    }
+    *out = &s;
+    return RSA_OK;
+}
+
+// 3-D tiled tensor map, 128-byte swizzle, zero fill out of bounds.
+bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t d0, uint64_t d1,
+           uint64_t d2, uint64_t pitch1, uint64_t pitch2, uint32_t box0, uint32_t box1) {
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {pitch1, pitch2};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, type, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Input tensor [BH][L][d] bf16, box of 64 columns x `rows` rows.
+bool map_input(CUtensorMap *m, const void *base, const Plan &p, uint32_t rows) {
+    return map3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, p.d, p.L, p.BH, uint64_t(p.d) * 2,
+                 uint64_t(p.L) * p.d * 2, 64, rows);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+SlabArgs slab_args(const Plan &p, const Group &G, int *status) {
+    SlabArgs a{};
+    a.L = p.L, a.Lp = p.Lp, a.N = p.N, a.c = p.c, a.causal = p.causal, a.d = p.d;
+    a.bh0 = G.bh0, a.nh = G.nh, a.r0 = G.r0, a.R = G.R;
+    a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(p.d)));
+    a.nRT = (G.R + 127) / 128;
+    a.status = status;
+    return a;
+}
+
+#define RSA_TRY(expr)                            \
+    do {                                         \
+        if ((expr) != cudaSuccess) return RSA_ERR_CUDA; \
+    } while (0)
+
+rsa_status_t check_common(const Plan &p, void *ws, size_t ws_bytes) {
+    if (p.total > ws_bytes) return RSA_ERR_WORKSPACE;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return RSA_ERR_INVALID_ARG;
+    return RSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *rsa_status_string(rsa_status_t s) {
+    switch (s) {
+        case RSA_OK: return "RSA_OK";
+        case RSA_ERR_INVALID_ARG: return "RSA_ERR_INVALID_ARG";
+        case RSA_ERR_UNSUPPORTED: return "RSA_ERR_UNSUPPORTED";
+        case RSA_ERR_WORKSPACE: return "RSA_ERR_WORKSPACE";
+        case RSA_ERR_CUDA: return "RSA_ERR_CUDA";
+        case RSA_ERR_TIMEOUT: return "RSA_ERR_TIMEOUT";
+    }
+    return "RSA_ERR_UNKNOWN";
+}
+
+size_t rsa_workspace_size(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                          int for_backward, size_t budget_bytes) {
+    rsa_status_t why;
+    if (!args_ok(B, H, L, d, N, dt, &why)) return 0;
+    const Plan p = make_plan(B, H, L, d, N, causal, dt, for_backward,
+                             budget_bytes ? budget_bytes : kDefaultBudget);
+    return p.total;
+}
+
+rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
+                               int for_backward, size_t ws_bytes, long long out[5]) {
+    rsa_status_t why;
+    if (!out) return RSA_ERR_INVALID_ARG;
+    if (!args_ok(B, H, L, d, N, dt, &why)) return why;
+    const Plan p = make_plan(B, H, L, d, N, causal, dt, for_backward, ws_bytes);
+    out[0] = p.ngroups;
+    out[1] = p.whole ? p.Gh : 1;
+    out[2] = p.R;
+    out[3] = p.Lp;
+    out[4] = static_cast<long long>(p.total);
+    return p.total > ws_bytes ? RSA_ERR_WORKSPACE : RSA_OK;
+}
+
+rsa_status_t rsa_last_device_status(void *stream) {
+    DeviceState *s = nullptr;
+    rsa_status_t st = device_state(&s);
+    if (st != RSA_OK) return st;
+    RSA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int v = 0;
+    RSA_TRY(cudaMemcpy(&v, s->status, sizeof(int), cudaMemcpyDeviceToHost));
+    const int zero = 0;
+    RSA_TRY(cudaMemcpy(s->status, &zero, sizeof(int), cudaMemcpyHostToDevice));
+    return static_cast<rsa_status_t>(v);
+}
+
+rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, float *lse, int B,
+                         int H, int L, int d, int N, int causal, rsa_dtype_t dt, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    rsa_status_t why;
+    if (!args_ok(B, H, L, d, N, dt, &why)) return why;
+    if (!Q || !K || !V || !O || !lse) return RSA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(lse))
+        return RSA_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, H, L, d, N, causal, dt, 0, ws_bytes);
+    rsa_status_t st = check_common(p, workspace, ws_bytes);
+    if (st != RSA_OK) return st;
+    DeviceState *dev = nullptr;
+    st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *slab = static_cast<float *>(workspace);
+
+    if (dt == RSA_F32) {
+        for (long long g = 0; g < p.ngroups; ++g) {
+            const Group G = group_of(p, g);
+            SlabArgs a = slab_args(p, G, dev->status);
+            RSA_TRY(rsa::launch_f32_qk_slab(static_cast<const float *>(Q),
+                                            static_cast<const float *>(K), slab, a, s));
+            RSA_TRY(rsa::launch_slab_softmax(slab, lse, a, 0, s));
+            a.scale = 1.f;
+            RSA_TRY(rsa::launch_f32_ring_rows(slab, static_cast<const float *>(V),
+                                              static_cast<float *>(O), a, s));
+        }
+        return RSA_OK;
+    }
+
+    CUtensorMap mQ, mK, mV;
+    if (!map_input(&mQ, Q, p, 128) || !map_input(&mK, K, p, 256) || !map_input(&mV, V, p, 64))
+        return RSA_ERR_CUDA;
+    for (long long g = 0; g < p.ngroups; ++g) {
+        const Group G = group_of(p, g);
+        SlabArgs a = slab_args(p, G, dev->status);
+        const uint64_t pitch = uint64_t(p.Lp) * 4;  // fp32 row; P (bf16) in its first half
+        CUtensorMap mS, mP;
+        if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
+                   pitch * G.R, 32, 32) ||
+            !map3d(&mP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, slab, p.Lp, G.R, G.nh, pitch,
+                   pitch * G.R, 64, 128))
+            return RSA_ERR_CUDA;
+        // ring pass 1: score slab
+        a.nCT = (p.Lp + 255) / 256;
+        a.ntiles = G.nh * a.nRT * a.nCT;
+        RSA_TRY(rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
+        // row softmax over the full key length
+        RSA_TRY(rsa::launch_slab_softmax(slab, lse, a, 1, s));
+        // ring pass 2: O = P V
+        a.nCT = 0;
+        a.ntiles = G.nh * a.nRT;
+        a.scale = 1.f;
+        RSA_TRY(rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
+    }
+    return RSA_OK;
+}
+
+rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const void *O,
+                          const void *dO, const float *lse, void *dQ, void *dK, void *dV, int B,
+                          int H, int L, int d, int N, int causal, rsa_dtype_t dt, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    rsa_status_t why;
+    if (!args_ok(B, H, L, d, N, dt, &why)) return why;
+    const void *ptrs[] = {Q, K, V, O, dO, lse, dQ, dK, dV};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return RSA_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, H, L, d, N, causal, dt, 1, ws_bytes);
+    rsa_status_t st = check_common(p, workspace, ws_bytes);
+    if (st != RSA_OK) return st;
+    DeviceState *dev = nullptr;
+    st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *Dvec = reinterpret_cast<float *>(ws + p.off_D);
+    const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
+
+    // D_i = dO_i . O_i
+    RSA_TRY(rsa::launch_rowdot(dO, O, Dvec, p.BH * L, d, dt == RSA_BF16, s));
+
+    if (dt == RSA_F32) {
+        for (long long g = 0; g < p.ngroups; ++g) {
+            const Group G = group_of(p, g);
+            SlabArgs a = slab_args(p, G, dev->status);
+            float *P = reinterpret_cast<float *>(ws);
+            float *dS = P + size_t(G.nh) * G.R * p.Lp;
+            const float *q = static_cast<const float *>(Q), *k = static_cast<const float *>(K);
+            RSA_TRY(rsa::launch_f32_bwd_slab(q, k, static_cast<const float *>(dO),
+                                             static_cast<const float *>(V), lse, Dvec, P, dS, a, s));
+            const int accum = G.first_of_head ? 0 : 1;
+            RSA_TRY(rsa::launch_f32_ring_keys(P, static_cast<const float *>(dO),
+                                              static_cast<float *>(dV), 1.f, accum, a, s));
+            RSA_TRY(rsa::launch_f32_ring_keys(dS, q, static_cast<float *>(dK), scale, accum, a, s));
+            a.scale = scale;
+            RSA_TRY(rsa::launch_f32_ring_rows(dS, k, static_cast<float *>(dQ), a, s));
+        }
+        return RSA_OK;
+    }
+
+    CUtensorMap mQk, mKk, mdOk, mVk, mKmn, mdOmn, mQmn;
+    if (!map_input(&mQk, Q, p, 128) || !map_input(&mKk, K, p, 128) ||
+        !map_input(&mdOk, dO, p, 128) || !map_input(&mVk, V, p, 128) ||
+        !map_input(&mKmn, K, p, 64) || !map_input(&mdOmn, dO, p, 64) ||
+        !map_input(&mQmn, Q, p, 64))
+        return RSA_ERR_CUDA;
+    float *acc_dK = p.whole ? nullptr : reinterpret_cast<float *>(ws + p.off_acc);
+    float *acc_dV = p.whole ? nullptr
+                            : reinterpret_cast<float *>(ws + p.off_acc +
+                                                        align_up(size_t(L) * d * 4, kAlign));
+    for (long long g = 0; g < p.ngroups; ++g) {
+        const Group G = group_of(p, g);
+        SlabArgs a = slab_args(p, G, dev->status);
+        const uint64_t pitch = uint64_t(p.Lp) * 2;
+        const size_t region = size_t(G.nh) * G.R * pitch;  // a multiple of 128 bytes
+        uint8_t *Pb = ws;
+        uint8_t *dSb = ws + region;
+        CUtensorMap mPst, mdSst, mPt, mdSt, mdSk;
+        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        if (!map3d(&mPst, bf, Pb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 32) ||
+            !map3d(&mdSst, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 32) ||
+            !map3d(&mPt, bf, Pb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 64) ||
+            !map3d(&mdSt, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 64) ||
+            !map3d(&mdSk, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 128))
+            return RSA_ERR_CUDA;
+        // P = exp(scale Q K^T - lse) and dS = P (dO V^T - D), as bf16 slabs
+        a.nCT = (p.Lp + 127) / 128;
+        a.ntiles = G.nh * a.nRT * a.nCT;
+        RSA_TRY(rsa::launch_bwd_slab(mQk, mKk, mdOk, mVk, mPst, mdSst, lse, Dvec, a, dev->sms, s));
+        // dV_m, dK_m gathered from every query chunk (key-major ring)
+        if (!p.whole && G.first_of_head) {
+            RSA_TRY(cudaMemsetAsync(acc_dK, 0, size_t(L) * d * 4, s));
+            RSA_TRY(cudaMemsetAsync(acc_dV, 0, size_t(L) * d * 4, s));
+        }
+        a.mode = p.whole ? 0 : (G.last_of_head ? 2 : 1);
+        a.nCT = 0;
+        a.ntiles = G.nh * ((L + 127) / 128);
+        RSA_TRY(rsa::launch_ring_keys(mPt, mdOmn, mdSt, mQmn, dK, dV, acc_dK, acc_dV, a, dev->sms, s));
+        // dQ_n = scale * sum_s dS_n[:, block m] K_m
+        a.mode = 0;
+        a.ntiles = G.nh * a.nRT;
+        RSA_TRY(rsa::launch_ring_rows(mdSk, mKmn, dQ, a, dev->sms, s));
+    }
+    return RSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// rsa_internal.h -- shared declarations between the C-ABI front end and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rsa {
+
+// One group of the slab schedule: heads [bh0, bh0 + nh) and, inside each of them, the query
+// rows [r0, r0 + R). The group's score slab lives in the workspace as [nh][R][Lp].
+struct Group {
+    int bh0, nh;
+    int r0, R;
+    int first_of_head;  // row-range groups: this group starts a head
+    int last_of_head;   // row-range groups: this group ends a head
+};
+
+// Arguments every slab kernel shares.
+struct SlabArgs {
+    int L, Lp, N, c, causal, d;
+    int bh0, nh, r0, R;
+    float scale;
+    int nRT;     // 128-row tiles per head in the group
+    int nCT;     // column tiles per head (kernel-specific width)
+    int ntiles;  // tiles in the launch (before causal skipping)
+    int mode;    // kernel-specific (see each kernel)
+    int *status; // device status word
+};
+
+// ---- bf16 tensor-core kernels (kernels_tc.cu) -------------------------------------------
+// Each returns a cudaError_t of its launch.
+cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mS,
+                           const SlabArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
+                             const SlabArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_bwd_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mdO,
+                            const CUtensorMap &mV, const CUtensorMap &mP, const CUtensorMap &mdS,
+                            const float *lse, const float *Dvec, const SlabArgs &a, int num_sms,
+                            cudaStream_t st);
+cudaError_t launch_ring_keys(const CUtensorMap &mPt, const CUtensorMap &mdO,
+                             const CUtensorMap &mdSt, const CUtensorMap &mQ, void *dK, void *dV,
+                             float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
+                             cudaStream_t st);
+cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
+
+// ---- CUDA-core kernels (kernels_simt.cu) -----------------------------------------------
+// Row softmax of the group's fp32 slab, in place: P written as bf16 (p_bf16 = 1) into the
+// first half of each fp32 row, or as fp32 over S (p_bf16 = 0). Writes lse.
+cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int p_bf16,
+                                cudaStream_t st);
+// D_i = dO_i . O_i for all rows of all heads (fp32 result).
+cudaError_t launch_rowdot(const void *dO, const void *O, float *Dvec, long long rows, int d,
+                          int bf16, cudaStream_t st);
+// fp32 path (every step in fp32 FMA).
+cudaError_t launch_f32_qk_slab(const float *Q, const float *K, float *S, const SlabArgs &a,
+                               cudaStream_t st);
+cudaError_t launch_f32_ring_rows(const float *A, const float *Bm, float *out, const SlabArgs &a,
+                                 cudaStream_t st);
+cudaError_t launch_f32_bwd_slab(const float *Q, const float *K, const float *dO, const float *V,
+                                const float *lse, const float *Dvec, float *P, float *dS,
+                                const SlabArgs &a, cudaStream_t st);
+cudaError_t launch_f32_ring_keys(const float *A, const float *Bm, float *out, float alpha,
+                                 int accumulate, const SlabArgs &a, cudaStream_t st);
+
+}  // namespace rsa

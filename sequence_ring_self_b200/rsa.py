@@ -1,0 +1,212 @@
+"""Python binding of the Ring Self-Attention C ABI (``include/rsa.h``).
+
+Argument marshalling only: tensors are checked for shape, dtype, device and layout, and their
+device pointers, sizes and the current CUDA stream are passed to the library; every step of
+the computation runs in the library's kernels. PyTorch supplies device memory and streams.
+There is no fallback: if the CUDA library is missing or the GPU is not sm_100, calls raise.
+
+Method: "Sequence Parallelism: Making 4D Parallelism Possible" (Li, Xue et al., 2021; review
+page, Abstract and "Proposed method"): the sequence is cut into N chunks, each chunk's score
+slab is built over a ring of key chunks, normalised by a full-row softmax, and multiplied
+with the values over a second ring pass; the backward pass runs the same ring.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "librsa_b200.so")
+
+RSA_OK, RSA_ERR_INVALID_ARG, RSA_ERR_UNSUPPORTED, RSA_ERR_WORKSPACE, RSA_ERR_CUDA, RSA_ERR_TIMEOUT = range(6)
+RSA_F32, RSA_BF16 = 0, 1
+
+EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
+            "rsa_last_device_status", "rsa_plan_describe")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class RSAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+def load_library(path: str | None = None):
+    """Load the CUDA library (it must have been built; see ``sequence_ring_self_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise ImportError(f"Ring Self-Attention CUDA library not built: {p} is missing "
+                              "(run `python -m sequence_ring_self_b200.build`)")
+        lib = ctypes.CDLL(p)
+        vp, sz, i = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        lib.rsa_workspace_size.argtypes = [i, i, i, i, i, i, i, i, sz]
+        lib.rsa_workspace_size.restype = sz
+        lib.rsa_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+        lib.rsa_forward.restype = i
+        lib.rsa_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz,
+                                     vp]
+        lib.rsa_backward.restype = i
+        lib.rsa_status_string.argtypes = [i]
+        lib.rsa_status_string.restype = ctypes.c_char_p
+        lib.rsa_last_device_status.argtypes = [vp]
+        lib.rsa_last_device_status.restype = i
+        lib.rsa_plan_describe.argtypes = [i, i, i, i, i, i, i, i, sz, ctypes.POINTER(ctypes.c_longlong)]
+        lib.rsa_plan_describe.restype = i
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().rsa_status_string(int(code)).decode()
+
+
+def _dtype_code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return RSA_BF16
+    if dtype == torch.float32:
+        return RSA_F32
+    raise TypeError(f"unsupported dtype {dtype}; use torch.bfloat16 or torch.float32")
+
+
+def workspace_size(B: int, H: int, L: int, d: int, N: int, causal: bool, dtype: torch.dtype,
+                   for_backward: bool, budget_bytes: int = 0) -> int:
+    """Workspace bytes for the plan that fits ``budget_bytes`` (0: the default plan)."""
+    n = load_library().rsa_workspace_size(B, H, L, d, N, int(bool(causal)), _dtype_code(dtype),
+                                          int(bool(for_backward)), int(budget_bytes))
+    if n == 0:
+        raise RSAError(RSA_ERR_INVALID_ARG, "rsa_workspace_size")
+    return int(n)
+
+
+def plan_describe(B: int, H: int, L: int, d: int, N: int, causal: bool, dtype: torch.dtype,
+                  for_backward: bool, ws_bytes: int) -> dict:
+    out = (ctypes.c_longlong * 5)()
+    rc = load_library().rsa_plan_describe(B, H, L, d, N, int(bool(causal)), _dtype_code(dtype),
+                                          int(bool(for_backward)), int(ws_bytes), out)
+    if rc not in (RSA_OK, RSA_ERR_WORKSPACE):
+        raise RSAError(rc, "rsa_plan_describe")
+    return {"groups": out[0], "heads_per_group": out[1], "rows_per_group": out[2],
+            "padded_row": out[3], "bytes": out[4], "fits": rc == RSA_OK}
+
+
+def last_device_status(stream: torch.cuda.Stream | None = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(load_library().rsa_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def _check_qkv(*ts):
+    q = ts[0]
+    if q.dim() != 4:
+        raise ValueError("tensors must be [B, H, L, d]")
+    for t in ts:
+        if t.shape != q.shape or t.dtype != q.dtype or t.device != q.device:
+            raise ValueError("Q, K, V (and O, dO) must share shape, dtype and device")
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, L, d]")
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is None:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError("workspace too small or not on the device")
+    return workspace
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward(q, k, v, N: int, causal: bool = False, *, ws_budget: int = 0, workspace=None,
+            out=None, lse=None, stream: torch.cuda.Stream | None = None):
+    """Ring Self-Attention forward. Returns (O [B,H,L,d] in the input dtype, lse [B,H,L] fp32)."""
+    _check_qkv(q, k, v)
+    B, H, L, d = q.shape
+    dt = _dtype_code(q.dtype)
+    lib = load_library()
+    nbytes = lib.rsa_workspace_size(B, H, L, d, N, int(bool(causal)), dt, 0, int(ws_budget))
+    if nbytes == 0:
+        raise RSAError(RSA_ERR_INVALID_ARG, "rsa_forward")
+    ws = _workspace(nbytes, q.device, workspace)
+    o = torch.empty_like(q) if out is None else out
+    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib.rsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
+                         int(bool(causal)), dt, _ptr(ws), ws.numel() * ws.element_size(),
+                         ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_forward")
+    return o, ls
+
+
+def backward(q, k, v, o, do, lse, N: int, causal: bool = False, *, ws_budget: int = 0,
+             workspace=None, dq=None, dk=None, dv=None, stream: torch.cuda.Stream | None = None):
+    """Ring Self-Attention backward. Returns (dQ, dK, dV) in the input dtype."""
+    _check_qkv(q, k, v, o, do)
+    B, H, L, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, L) or not lse.is_contiguous():
+        raise ValueError("lse must be contiguous fp32 [B, H, L]")
+    dt = _dtype_code(q.dtype)
+    lib = load_library()
+    nbytes = lib.rsa_workspace_size(B, H, L, d, N, int(bool(causal)), dt, 1, int(ws_budget))
+    if nbytes == 0:
+        raise RSAError(RSA_ERR_INVALID_ARG, "rsa_backward")
+    ws = _workspace(nbytes, q.device, workspace)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib.rsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                          _ptr(dk), _ptr(dv), B, H, L, d, N, int(bool(causal)), dt, _ptr(ws),
+                          ws.numel() * ws.element_size(), ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_backward")
+    return dq, dk, dv
+
+
+class RingSelfAttention(torch.autograd.Function):
+    """autograd wrapper: ``RingSelfAttention.apply(q, k, v, N, causal)`` -> O."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, N, causal=False):
+        o, lse = forward(q, k, v, N, causal)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.N, ctx.causal = N, causal
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, ctx.N, ctx.causal)
+        return dq, dk, dv, None, None
+
+
+def forward_backward_host(q, k, v, do, N: int, causal: bool = False, *, ws_budget: int = 0,
+                          device=None, results=None):
+    """One forward + backward from host (ideally pinned) tensors: copies Q, K, V, dO to the
+    device, runs the library's forward and backward there, and copies O, lse, dQ, dK, dV
+    back into host tensors (``results`` if given, a dict of pinned tensors by name)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in (q, k, v, do))
+    o, lse = forward(qd, kd, vd, N, causal, ws_budget=ws_budget)
+    dq, dk, dv = backward(qd, kd, vd, o, dod, lse, N, causal, ws_budget=ws_budget)
+    names = ("O", "lse", "dQ", "dK", "dV")
+    if results is None:
+        results = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                   for n, t in zip(names, (o, lse, dq, dk, dv))}
+    for n, t in zip(names, (o, lse, dq, dk, dv)):
+        results[n].copy_(t, non_blocking=True)
+    return results

@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function
+``include/rsa.h`` declares, rejects bad arguments before launching anything, and plans its
+workspace consistently."""
+import os
+import re
+
+import pytest
+import torch
+
+from sequence_ring_self_b200 import build, rsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return rsa.load_library()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "rsa.h")).read()
+    return re.findall(r"RSA_API\s+[\w\s\*]+?\b(rsa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_abi():
+    assert sorted(_declared()) == sorted(rsa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert rsa.status_string(rsa.RSA_OK) == "RSA_OK"
+    assert rsa.status_string(rsa.RSA_ERR_WORKSPACE) == "RSA_ERR_WORKSPACE"
+    assert rsa.status_string(99) == "RSA_ERR_UNKNOWN"
+
+
+FAKE = 0x100000  # a 16-byte-aligned non-null pointer that is never dereferenced
+
+
+def _fwd(lib, B=1, H=1, L=128, d=64, N=1, dt=rsa.RSA_BF16, ptr=FAKE, ws=FAKE, ws_bytes=1 << 30,
+         lse=FAKE):
+    return lib.rsa_forward(ptr, ptr, ptr, ptr, lse, B, H, L, d, N, 0, dt, ws, ws_bytes, None)
+
+
+def _bwd(lib, B=1, H=1, L=128, d=64, N=1, dt=rsa.RSA_BF16, ptr=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return lib.rsa_backward(ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, B, H, L, d, N, 0, dt, ws,
+                            ws_bytes, None)
+
+
+@pytest.mark.parametrize("call", [_fwd, _bwd])
+def test_argument_errors_are_reported_before_any_launch(lib, call):
+    assert call(lib, L=100, N=3) == rsa.RSA_ERR_INVALID_ARG          # L % N != 0
+    assert call(lib, B=0) == rsa.RSA_ERR_INVALID_ARG
+    assert call(lib, N=0) == rsa.RSA_ERR_INVALID_ARG
+    assert call(lib, L=-4) == rsa.RSA_ERR_INVALID_ARG
+    assert call(lib, d=96) == rsa.RSA_ERR_UNSUPPORTED                # bf16 head dim
+    assert call(lib, d=128, dt=rsa.RSA_F32) == rsa.RSA_ERR_UNSUPPORTED
+    assert call(lib, dt=7) == rsa.RSA_ERR_UNSUPPORTED
+    assert call(lib, ptr=0) == rsa.RSA_ERR_INVALID_ARG               # null
+    assert call(lib, ptr=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG        # misaligned
+    assert call(lib, ws_bytes=1024) == rsa.RSA_ERR_WORKSPACE         # too small
+    assert call(lib, ws=FAKE + 64) == rsa.RSA_ERR_INVALID_ARG        # workspace not 256-aligned
+    assert call(lib, ws=0) == rsa.RSA_ERR_INVALID_ARG
+
+
+def test_forward_rejects_null_lse(lib):
+    assert _fwd(lib, lse=0) == rsa.RSA_ERR_INVALID_ARG
+
+
+def test_workspace_size_invalid_is_zero(lib):
+    assert lib.rsa_workspace_size(1, 1, 100, 64, 3, 0, rsa.RSA_BF16, 0, 0) == 0
+    assert lib.rsa_workspace_size(1, 1, 128, 80, 1, 0, rsa.RSA_BF16, 0, 0) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("bwd", [False, True])
+def test_plans_fit_their_budget_and_grow_with_it(lib, dtype, bwd):
+    d = 64
+    B, H, L, N = 2, 3, 1000, 8
+    sizes = []
+    for budget in [1, 1 << 18, 1 << 20, 1 << 22, 1 << 24, 1 << 26, 1 << 30]:
+        n = rsa.workspace_size(B, H, L, d, N, False, dtype, bwd, budget)
+        info = rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, n)
+        assert info["fits"] and info["bytes"] == n
+        if n > budget:  # only the minimum plan may exceed the budget
+            assert info["rows_per_group"] == 128 and info["heads_per_group"] == 1
+        sizes.append(n)
+        Lp = info["padded_row"]
+        assert Lp % 64 == 0 and Lp >= L
+        rows = info["rows_per_group"]
+        assert rows == L or rows % 128 == 0
+        # every (head, row) is covered exactly once by the groups
+        if rows == L:
+            assert info["groups"] == -(-B * H // info["heads_per_group"])
+        else:
+            assert info["groups"] == B * H * -(-L // rows)
+    assert sizes == sorted(sizes)
+    assert rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, sizes[0] - 1)["fits"] is False
+
+
+def test_default_plan_is_capped_at_one_gib(lib):
+    n = rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, True, 0)
+    assert n <= (1 << 30)
+    info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, True, n)
+    assert info["fits"]

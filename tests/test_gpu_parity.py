@@ -1,0 +1,295 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on the same seeded
+inputs.
+
+Tolerances (fixed by the method's target precision): fp32 max-abs <= 1e-5; bf16 inputs with
+fp32 accumulation: max-abs <= 2e-2 and relative L2 <= 1e-2, on O, dQ, dK and dV.
+
+Workloads: the five transformer-shaped configurations of the method's evaluation (the pages
+quote only end-to-end results, so synthetic inputs of these shapes stand in), plus ragged,
+degenerate and sharp-attention edge cases. Large problems are compared on sampled heads, rows
+or keys that the oracle computes one by one, and through N-invariance (the ring result must
+not depend on the chunk count beyond rounding).
+"""
+import types
+
+import numpy as np
+import pytest
+import torch
+
+from sequence_ring_self_b200 import build, rsa
+from sequence_ring_self_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+F32_MAXABS = 1e-5
+BF16_MAXABS = 2e-2
+BF16_RELL2 = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    build.build()
+    rsa.load_library()
+    torch.cuda.set_device(0)
+
+
+def np64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_l2(a, b):
+    den = np.linalg.norm(b.ravel())
+    return np.linalg.norm((a - b).ravel()) / (den if den > 0 else 1.0)
+
+
+def check(got, ref, dtype, name):
+    err = np.abs(got - ref).max() if got.size else 0.0
+    if dtype == "f32":
+        assert err <= F32_MAXABS, f"{name}: max-abs {err:.3e} > {F32_MAXABS}"
+    else:
+        r = rel_l2(got, ref)
+        assert err <= BF16_MAXABS and r <= BF16_RELL2, f"{name}: max-abs {err:.3e}, rel-L2 {r:.3e}"
+
+
+def run(x, N, causal, *, bwd=True, ws_budget=0):
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+    o, lse = rsa.forward(q, k, v, N, causal, ws_budget=ws_budget)
+    out = {"O": o, "lse": lse}
+    if bwd:
+        dq, dk, dv = rsa.backward(q, k, v, o, do, lse, N, causal, ws_budget=ws_budget)
+        out.update(dQ=dq, dK=dk, dV=dv)
+    torch.cuda.synchronize()
+    assert rsa.last_device_status() == rsa.RSA_OK
+    return {n: np64(t) for n, t in out.items()}
+
+
+def check_full(orc, x, got, causal, bwd=True):
+    o, lse = orc.forward(x.q, x.k, x.v, causal)
+    check(got["O"], o, x.dtype, "O")
+    np.testing.assert_allclose(got["lse"], lse, rtol=0, atol=1e-5 if x.dtype == "f32" else 1e-3)
+    if bwd:
+        for name, ref in zip(("dQ", "dK", "dV"), orc.backward(x.q, x.k, x.v, x.do, causal)):
+            check(got[name], ref, x.dtype, name)
+
+
+def check_sampled(orc, x, got, causal, heads, rows, keys):
+    for (b, h) in heads:
+        o, lse = orc.forward_rows(x.q, x.k, x.v, b, h, rows, causal)
+        check(got["O"][b, h, rows], o, x.dtype, f"O[{b},{h}] rows")
+        np.testing.assert_allclose(got["lse"][b, h, rows], lse, rtol=0, atol=1e-3)
+        dq = orc.backward_rows(x.q, x.k, x.v, x.do, b, h, rows, causal)
+        check(got["dQ"][b, h, rows], dq, x.dtype, f"dQ[{b},{h}] rows")
+    if keys is not None:
+        b, h = heads[0]
+        dk, dv = orc.backward_keys(x.q, x.k, x.v, x.do, b, h, keys, causal)
+        check(got["dK"][b, h, keys], dk, x.dtype, f"dK[{b},{h}] keys")
+        check(got["dV"][b, h, keys], dv, x.dtype, f"dV[{b},{h}] keys")
+
+
+def sample(L, seed, n=60, edges=(0, 1)):
+    """Edge rows plus n seeded-random rows: the relative L2 over a sample stays representative
+    of the whole tensor (a handful of hand-picked rows would be dominated by the few causal
+    rows that see only one or two keys, where the bf16 rounding of P and O does not average)."""
+    rng = np.random.default_rng(seed)
+    picks = set(rng.choice(L, size=min(n, L), replace=False).tolist())
+    picks |= {e % L for e in edges} | {L - 1, L - 2 if L > 1 else 0}
+    return sorted(picks)
+
+
+def check_invariants(x, got):
+    """Properties of the exact result that hold at any size: key gradients sum to zero over the
+    keys, value gradients sum to the output gradients (P is row-stochastic)."""
+    dk_sum = got["dK"].sum(axis=2)
+    dv_sum = got["dV"].sum(axis=2)
+    scale_k = np.abs(got["dK"]).sum(axis=2) + 1e-30
+    assert np.all(np.abs(dk_sum) <= 2e-2 * scale_k + 1e-6)
+    do_sum = x.do.sum(axis=2)
+    assert rel_l2(dv_sum, do_sum) <= 1e-2
+
+
+# ------------------------------------------------------------------ the five configurations
+
+def test_config1_fp32_forward(orc):
+    """B=1 H=2 L=256 d=32 N=4 fp32, N(0,1), seed 0; vs oracle and vs the unchunked run."""
+    x = make_inputs(1, 2, 256, 32, seed=0, dtype="f32")
+    got = run(x, 4, False, bwd=False)
+    check_full(orc, x, got, False, bwd=False)
+    o_ring, _ = orc.forward_ring(x.q, x.k, x.v, 4)
+    check(got["O"], o_ring, "f32", "O vs ring oracle")
+    got1 = run(x, 1, False, bwd=False)
+    check(got["O"], got1["O"], "f32", "O(N=4) vs O(N=1)")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_config1_fp32_backward(orc, causal):
+    x = make_inputs(1, 2, 256, 32, seed=0, dtype="f32")
+    got = run(x, 4, causal)
+    check_full(orc, x, got, causal)
+
+
+def test_config2_bert_base(orc):
+    """B=8 H=12 L=512 d=64 N=4 bf16, N(0,1)/sqrt(d), dO ~ N(0,1), non-causal, full tensors."""
+    x = make_inputs(8, 12, 512, 64, seed=2, dtype="bf16")
+    got = run(x, 4, False)
+    check_full(orc, x, got, False)
+    check_invariants(x, got)
+
+
+def test_config3_gpt_causal(orc):
+    """B=4 H=16 L=4096 d=64 N=8 bf16 causal; four sampled heads compared in full."""
+    x = make_inputs(4, 16, 4096, 64, seed=3, dtype="bf16")
+    got = run(x, 8, True)
+    heads = [(0, 0), (3, 15), (1, 7), (2, 10)]
+    sub = types.SimpleNamespace(dtype="bf16")
+    for n in ("q", "k", "v", "do"):
+        setattr(sub, n, np.stack([getattr(x, n)[b, h] for b, h in heads])[None])
+    g = {n: np.stack([got[n][b, h] for b, h in heads])[None] for n in got}
+    check_full(orc, sub, g, True)
+    check_invariants(x, got)
+
+
+def test_config4_long_sequence(orc):
+    """B=1 H=16 L=16384 d=128 N=16 bf16, slab groups in sequence (1 GiB default workspace):
+    sampled rows of two heads and sampled keys of one head."""
+    x = make_inputs(1, 16, 16384, 128, seed=4, dtype="bf16")
+    info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, True,
+                             rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, True))
+    assert info["groups"] > 1  # the slab is processed group by group
+    got = run(x, 16, False)
+    rows = sample(16384, 4, edges=(0, 1, 1023, 1024))
+    check_sampled(orc, x, got, False, [(0, 0), (0, 13)], rows, keys=sample(16384, 40, n=24))
+    check_invariants(x, got)
+
+
+SWEEP_L = [1024, 2048, 4096, 8192]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("L", SWEEP_L)
+def test_sweep_against_oracle_and_n_invariance(orc, L, causal):
+    """B=1 H=16 d=64 bf16: every N in {1,2,4,8,16} agrees with N=1; the oracle checks one head."""
+    idx = SWEEP_L.index(L) * 10 + int(causal)
+    x = make_inputs(1, 16, L, 64, seed=5 + idx, dtype="bf16")
+    base = run(x, 1, causal)
+    for N in (2, 4, 8, 16):
+        got = run(x, N, causal)
+        for n in ("O", "dQ", "dK", "dV"):
+            check(got[n], base[n], "bf16", f"{n} N={N} vs N=1")
+    got = run(x, 16, causal)
+    check_sampled(orc, x, got, causal, [(0, 5)], sample(L, idx), keys=sample(L, 100 + idx, n=24))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sweep_maximum_length(orc, causal):
+    """The sweep's largest point, L = 32768, N = 16: sampled rows against the oracle."""
+    x = make_inputs(1, 16, 32768, 64, seed=60 + int(causal), dtype="bf16")
+    got = run(x, 16, causal)
+    check_sampled(orc, x, got, causal, [(0, 3)], sample(32768, 7, edges=(0, 77, 16384)), keys=None)
+    check_invariants(x, got)
+
+
+# ------------------------------------------------------------------ edge cases
+
+EDGE = [  # (B, H, L, d, N)
+    (1, 1, 1, 64, 1),      # one token
+    (1, 2, 50, 64, 5),     # smaller than one tile, ragged
+    (2, 1, 130, 64, 2),    # one full 128-row tile plus a 2-row tail
+    (1, 3, 200, 128, 4),   # d = 128, ragged chunks (c = 50)
+    (1, 2, 320, 64, 5),    # c = 64
+    (1, 1, 700, 128, 7),   # several tiles, ragged tail, c = 100
+    (3, 1, 384, 64, 384),  # one row per chunk
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", EDGE)
+def test_edge_shapes_bf16(orc, shape, causal):
+    B, H, L, d, N = shape
+    x = make_inputs(B, H, L, d, seed=100 + L + d, dtype="bf16")
+    got = run(x, N, causal)
+    check_full(orc, x, got, causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 32, 1), (1, 2, 70, 32, 7), (2, 1, 200, 64, 4),
+                                   (1, 1, 333, 64, 3)])
+def test_edge_shapes_f32(orc, shape, causal):
+    B, H, L, d, N = shape
+    x = make_inputs(B, H, L, d, seed=200 + L, dtype="f32")
+    got = run(x, N, causal)
+    check_full(orc, x, got, causal)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_range_groups(orc, dtype, causal):
+    """A small workspace budget forces groups of 128-row ranges of one head (the last one
+    ragged), with dK/dV accumulated across groups."""
+    d = 64
+    B, H, L, N = 1, 2, 700, 7
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    budget = 300 * 1024
+    info = rsa.plan_describe(B, H, L, d, N, causal, tdt, True,
+                             rsa.workspace_size(B, H, L, d, N, causal, tdt, True, budget))
+    assert info["rows_per_group"] < L and info["groups"] > B * H
+    x = make_inputs(B, H, L, d, seed=300 + int(causal), dtype=dtype)
+    got = run(x, N, causal, ws_budget=budget)
+    check_full(orc, x, got, causal)
+    whole = run(x, N, causal)
+    for n in ("O", "dQ", "dK", "dV"):
+        check(got[n], whole[n], dtype, f"{n} row groups vs whole heads")
+
+
+@pytest.mark.parametrize("kind", ["unscaled", "sharp"])
+def test_sharp_attention(orc, kind):
+    """Score std ~1 (unscaled inputs) and sharp rows (Q x 8): a wrong scale or a missing
+    max-subtraction would show here, not at the configurations' near-uniform attention."""
+    extra = 8.0 if kind == "sharp" else 1.0
+    x = make_inputs(2, 2, 512, 64, seed=400 + int(extra), dtype="bf16", qkv_scale=1.0,
+                    q_extra_scale=extra)
+    for causal in (False, True):
+        got = run(x, 4, causal)
+        check_full(orc, x, got, causal)
+        o, _ = orc.forward(x.q, x.k, x.v, causal)
+        assert rel_l2(got["O"], o) <= BF16_RELL2
+
+
+def test_deterministic_and_stream_ordered():
+    x = make_inputs(2, 4, 1000, 64, seed=7, dtype="bf16")
+    a = run(x, 8, True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run(x, 8, True)
+    for n in a:
+        np.testing.assert_array_equal(a[n], b[n])
+
+
+def test_autograd_wrapper_and_host_api(orc):
+    x = make_inputs(1, 2, 256, 64, seed=8, dtype="bf16")
+    dev = torch.device("cuda", 0)
+    q, k, v = (x.torch(n, dev).requires_grad_() for n in ("q", "k", "v"))
+    o = rsa.RingSelfAttention.apply(q, k, v, 4, True)
+    o.backward(x.torch("do", dev))
+    ref = run(x, 4, True)
+    np.testing.assert_array_equal(np64(o), ref["O"])
+    for t, n in ((q, "dQ"), (k, "dK"), (v, "dV")):
+        np.testing.assert_array_equal(np64(t.grad), ref[n])
+    host = {n: x.torch(n).pin_memory() for n in ("q", "k", "v", "do")}
+    res = rsa.forward_backward_host(host["q"], host["k"], host["v"], host["do"], 4, True)
+    torch.cuda.synchronize()
+    for n in ("O", "lse", "dQ", "dK", "dV"):
+        np.testing.assert_array_equal(res[n].to(torch.float64).numpy(), ref[n])
+
+
+def test_library_errors_raise():
+    dev = torch.device("cuda", 0)
+    q = torch.zeros(1, 1, 100, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(rsa.RSAError):
+        rsa.forward(q, q, q, 3)
+    small = torch.empty(1024, dtype=torch.uint8, device=dev)
+    q2 = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(ValueError):
+        rsa.forward(q2, q2, q2, 1, workspace=small)
