@@ -119,6 +119,20 @@ RSA_API rsa_status_t rsa_last_device_status(void *stream);
 RSA_API rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
                                int for_backward, size_t ws_bytes, long long out[5]);
 
+/*
+ * Per-kernel timing, for benchmarks. While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the launch's stream (an extra ~1 us per launch);
+ * rsa_profile_read() waits for those events, adds their elapsed times per kernel kind into
+ * ms[kind] and the launch counts into launches[kind] (arrays of rsa_profile_kinds() entries,
+ * caller-owned, host memory), and forgets them. Events come from a pool owned by the
+ * library. Enabling or disabling drops unread records. Not for use during stream capture.
+ * Returns RSA_ERR_CUDA if an event call fails.
+ */
+RSA_API rsa_status_t rsa_profile_enable(int on);
+RSA_API int rsa_profile_kinds(void);
+RSA_API const char *rsa_profile_kind_name(int kind); /* NULL if out of range */
+RSA_API rsa_status_t rsa_profile_read(double *ms, long long *launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,6 +33,18 @@ def _deps():
             + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
+def source_digest() -> str:
+    """SHA-256 over the library's sources (identifies the kernels a profile was taken on)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(_deps()):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True

@@ -122,27 +122,44 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
+// D_i = dO_i . O_i. The flattened [rows][D] arrays are read as 16-byte vectors: vector t holds
+// elements [8t, 8t + 8) (bf16) or [4t, 4t + 4) (fp32), so TPR = D / (elements per vector)
+// consecutive threads share a row and reduce with shuffles. Warps stride in lockstep.
 template <int D, bool BF16>
-__global__ void rowdot_kernel(const void *__restrict__ dO, const void *__restrict__ O,
-                              float *__restrict__ Dvec, long long rows) {
-    const long long r = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+__global__ void __launch_bounds__(256)
+    rowdot_kernel(const uint4 *__restrict__ dO, const uint4 *__restrict__ O,
+                  float *__restrict__ Dvec, long long rows) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    constexpr int TPR = D / EPV;
+    const long long total = rows * TPR;
     const int lane = threadIdx.x & 31;
-    if (r >= rows) return;
-    constexpr int PER = D / 32;
-    float s = 0.f;
-    if (BF16) {
-        const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(dO) + r * D + lane * PER;
-        const __nv_bfloat16 *b = static_cast<const __nv_bfloat16 *>(O) + r * D + lane * PER;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long t0 = static_cast<long long>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+         t0 < total; t0 += stride) {
+        const long long t = t0 + lane;
+        float s = 0.f;
+        if (t < total) {
+            const uint4 a = dO[t], b = O[t];
+            if (BF16) {
+                const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+                const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
 #pragma unroll
-        for (int e = 0; e < PER; ++e) s += __bfloat162float(a[e]) * __bfloat162float(b[e]);
-    } else {
-        const float *a = static_cast<const float *>(dO) + r * D + lane * PER;
-        const float *b = static_cast<const float *>(O) + r * D + lane * PER;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 u = __bfloat1622float2(x[e]), w = __bfloat1622float2(y[e]);
+                    s = fmaf(u.x, w.x, s);
+                    s = fmaf(u.y, w.y, s);
+                }
+            } else {
+                const float *x = reinterpret_cast<const float *>(&a);
+                const float *y = reinterpret_cast<const float *>(&b);
 #pragma unroll
-        for (int e = 0; e < PER; ++e) s += a[e] * b[e];
+                for (int e = 0; e < 4; ++e) s = fmaf(x[e], y[e], s);
+            }
+        }
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (t < total && (lane % TPR) == 0) Dvec[t / TPR] = s;
     }
-    s = warp_sum(s);
-    if (lane == 0) Dvec[r] = s;
 }
 
 // ------------------------------------------------------------------------- fp32 path
@@ -409,15 +426,19 @@ cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int 
 
 cudaError_t launch_rowdot(const void *dO, const void *O, float *Dvec, long long rows, int d,
                           int bf16, cudaStream_t st) {
-    const long long grid = (rows + 7) / 8;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const long long vectors = rows * d / (bf16 ? 8 : 4);
+    long long grid = (vectors + 255) / 256;
+    if (grid > 148 * 16) grid = 148 * 16;
+    if (grid < 1) grid = 1;
     const unsigned g = static_cast<unsigned>(grid);
+    auto *a = static_cast<const uint4 *>(dO);
+    auto *b = static_cast<const uint4 *>(O);
     if (bf16) {
-        if (d == 64) rowdot_kernel<64, true><<<g, 256, 0, st>>>(dO, O, Dvec, rows);
-        else rowdot_kernel<128, true><<<g, 256, 0, st>>>(dO, O, Dvec, rows);
+        if (d == 64) rowdot_kernel<64, true><<<g, 256, 0, st>>>(a, b, Dvec, rows);
+        else rowdot_kernel<128, true><<<g, 256, 0, st>>>(a, b, Dvec, rows);
     } else {
-        if (d == 32) rowdot_kernel<32, false><<<g, 256, 0, st>>>(dO, O, Dvec, rows);
-        else rowdot_kernel<64, false><<<g, 256, 0, st>>>(dO, O, Dvec, rows);
+        if (d == 32) rowdot_kernel<32, false><<<g, 256, 0, st>>>(a, b, Dvec, rows);
+        else rowdot_kernel<64, false><<<g, 256, 0, st>>>(a, b, Dvec, rows);
     }
     return cudaGetLastError();
 }

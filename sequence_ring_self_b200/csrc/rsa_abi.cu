@@ -12,6 +12,7 @@
 #include <math.h>
 #include <mutex>
 #include <string.h>
+#include <vector>
 
 #include "../../include/rsa.h"
 #include "rsa_internal.h"
@@ -189,6 +190,70 @@ rsa_status_t device_state(DeviceState **out) {
     return RSA_OK;
 }
 
+// ---------------------------------------------------------------- per-kernel timing
+
+enum Kind {
+    K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_SLAB, K_RING_KEYS, K_DQ,
+    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_COUNT
+};
+const char *kKindNames[K_COUNT] = {
+    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_slab", "dkdv_ring_keys",
+    "dq_ring_rows", "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys",
+    "f32_dq_ring_rows"};
+
+struct ProfRec {
+    int kind;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mutex;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t pool_event() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void drop_records() {
+    for (auto &r : g_prof) {
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_prof.clear();
+}
+
+// Launch helper: brackets the launch with events when profiling is on.
+template <class F>
+rsa_status_t timed(int kind, cudaStream_t s, F &&launch) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (g_prof_on) {
+        std::lock_guard<std::mutex> lock(g_prof_mutex);
+        a = pool_event();
+        b = pool_event();
+        if (!a || !b || cudaEventRecord(a, s) != cudaSuccess) return RSA_ERR_CUDA;
+    }
+    if (launch() != cudaSuccess) return RSA_ERR_CUDA;
+    if (a) {
+        std::lock_guard<std::mutex> lock(g_prof_mutex);
+        if (cudaEventRecord(b, s) != cudaSuccess) return RSA_ERR_CUDA;
+        g_prof.push_back({kind, a, b});
+    }
+    return RSA_OK;
+}
+
+#define RSA_LAUNCH(kind, expr)                                                   \
+    do {                                                                         \
+        rsa_status_t st_ = timed(kind, s, [&]() -> cudaError_t { return (expr); }); \
+        if (st_ != RSA_OK) return st_;                                           \
+    } while (0)
+
 // 3-D tiled tensor map, 128-byte swizzle, zero fill out of bounds.
 bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t d0, uint64_t d1,
            uint64_t d2, uint64_t pitch1, uint64_t pitch2, uint32_t box0, uint32_t box1) {
@@ -270,6 +335,36 @@ rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rs
     return p.total > ws_bytes ? RSA_ERR_WORKSPACE : RSA_OK;
 }
 
+rsa_status_t rsa_profile_enable(int on) {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    drop_records();
+    g_prof_on = on != 0;
+    return RSA_OK;
+}
+
+int rsa_profile_kinds(void) { return K_COUNT; }
+
+const char *rsa_profile_kind_name(int kind) {
+    return kind >= 0 && kind < K_COUNT ? kKindNames[kind] : nullptr;
+}
+
+rsa_status_t rsa_profile_read(double *ms, long long *launches) {
+    if (!ms || !launches) return RSA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
+    rsa_status_t st = RSA_OK;
+    for (auto &r : g_prof) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+            st = RSA_ERR_CUDA;
+            continue;
+        }
+        ms[r.kind] += t;
+        launches[r.kind] += 1;
+    }
+    drop_records();
+    return st;
+}
+
 rsa_status_t rsa_last_device_status(void *stream) {
     DeviceState *s = nullptr;
     rsa_status_t st = device_state(&s);
@@ -303,11 +398,11 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         for (long long g = 0; g < p.ngroups; ++g) {
             const Group G = group_of(p, g);
             SlabArgs a = slab_args(p, G, dev->status);
-            RSA_TRY(rsa::launch_f32_qk_slab(static_cast<const float *>(Q),
+            RSA_LAUNCH(K_F32_QK, rsa::launch_f32_qk_slab(static_cast<const float *>(Q),
                                             static_cast<const float *>(K), slab, a, s));
-            RSA_TRY(rsa::launch_slab_softmax(slab, lse, a, 0, s));
+            RSA_LAUNCH(K_SOFTMAX, rsa::launch_slab_softmax(slab, lse, a, 0, s));
             a.scale = 1.f;
-            RSA_TRY(rsa::launch_f32_ring_rows(slab, static_cast<const float *>(V),
+            RSA_LAUNCH(K_F32_PV, rsa::launch_f32_ring_rows(slab, static_cast<const float *>(V),
                                               static_cast<float *>(O), a, s));
         }
         return RSA_OK;
@@ -329,14 +424,14 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         // ring pass 1: score slab
         a.nCT = (p.Lp + 255) / 256;
         a.ntiles = G.nh * a.nRT * a.nCT;
-        RSA_TRY(rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
+        RSA_LAUNCH(K_QK_SLAB, rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
         // row softmax over the full key length
-        RSA_TRY(rsa::launch_slab_softmax(slab, lse, a, 1, s));
+        RSA_LAUNCH(K_SOFTMAX, rsa::launch_slab_softmax(slab, lse, a, 1, s));
         // ring pass 2: O = P V
         a.nCT = 0;
         a.ntiles = G.nh * a.nRT;
         a.scale = 1.f;
-        RSA_TRY(rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
+        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
     }
     return RSA_OK;
 }
@@ -362,7 +457,7 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
     const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
 
     // D_i = dO_i . O_i
-    RSA_TRY(rsa::launch_rowdot(dO, O, Dvec, p.BH * L, d, dt == RSA_BF16, s));
+    RSA_LAUNCH(K_ROWDOT, rsa::launch_rowdot(dO, O, Dvec, p.BH * L, d, dt == RSA_BF16, s));
 
     if (dt == RSA_F32) {
         for (long long g = 0; g < p.ngroups; ++g) {
@@ -371,14 +466,14 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
             float *P = reinterpret_cast<float *>(ws);
             float *dS = P + size_t(G.nh) * G.R * p.Lp;
             const float *q = static_cast<const float *>(Q), *k = static_cast<const float *>(K);
-            RSA_TRY(rsa::launch_f32_bwd_slab(q, k, static_cast<const float *>(dO),
+            RSA_LAUNCH(K_F32_BWD, rsa::launch_f32_bwd_slab(q, k, static_cast<const float *>(dO),
                                              static_cast<const float *>(V), lse, Dvec, P, dS, a, s));
             const int accum = G.first_of_head ? 0 : 1;
-            RSA_TRY(rsa::launch_f32_ring_keys(P, static_cast<const float *>(dO),
+            RSA_LAUNCH(K_F32_KEYS, rsa::launch_f32_ring_keys(P, static_cast<const float *>(dO),
                                               static_cast<float *>(dV), 1.f, accum, a, s));
-            RSA_TRY(rsa::launch_f32_ring_keys(dS, q, static_cast<float *>(dK), scale, accum, a, s));
+            RSA_LAUNCH(K_F32_KEYS, rsa::launch_f32_ring_keys(dS, q, static_cast<float *>(dK), scale, accum, a, s));
             a.scale = scale;
-            RSA_TRY(rsa::launch_f32_ring_rows(dS, k, static_cast<float *>(dQ), a, s));
+            RSA_LAUNCH(K_F32_DQ, rsa::launch_f32_ring_rows(dS, k, static_cast<float *>(dQ), a, s));
         }
         return RSA_OK;
     }
@@ -411,7 +506,7 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
         // P = exp(scale Q K^T - lse) and dS = P (dO V^T - D), as bf16 slabs
         a.nCT = (p.Lp + 127) / 128;
         a.ntiles = G.nh * a.nRT * a.nCT;
-        RSA_TRY(rsa::launch_bwd_slab(mQk, mKk, mdOk, mVk, mPst, mdSst, lse, Dvec, a, dev->sms, s));
+        RSA_LAUNCH(K_BWD_SLAB, rsa::launch_bwd_slab(mQk, mKk, mdOk, mVk, mPst, mdSst, lse, Dvec, a, dev->sms, s));
         // dV_m, dK_m gathered from every query chunk (key-major ring)
         if (!p.whole && G.first_of_head) {
             RSA_TRY(cudaMemsetAsync(acc_dK, 0, size_t(L) * d * 4, s));
@@ -420,11 +515,11 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
         a.mode = p.whole ? 0 : (G.last_of_head ? 2 : 1);
         a.nCT = 0;
         a.ntiles = G.nh * ((L + 127) / 128);
-        RSA_TRY(rsa::launch_ring_keys(mPt, mdOmn, mdSt, mQmn, dK, dV, acc_dK, acc_dV, a, dev->sms, s));
+        RSA_LAUNCH(K_RING_KEYS, rsa::launch_ring_keys(mPt, mdOmn, mdSt, mQmn, dK, dV, acc_dK, acc_dV, a, dev->sms, s));
         // dQ_n = scale * sum_s dS_n[:, block m] K_m
         a.mode = 0;
         a.ntiles = G.nh * a.nRT;
-        RSA_TRY(rsa::launch_ring_rows(mdSk, mKmn, dQ, a, dev->sms, s));
+        RSA_LAUNCH(K_DQ, rsa::launch_ring_rows(mdSk, mKmn, dQ, a, dev->sms, s));
     }
     return RSA_OK;
 }

@@ -25,7 +25,8 @@ RSA_OK, RSA_ERR_INVALID_ARG, RSA_ERR_UNSUPPORTED, RSA_ERR_WORKSPACE, RSA_ERR_CUD
 RSA_F32, RSA_BF16 = 0, 1
 
 EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
-            "rsa_last_device_status", "rsa_plan_describe")
+            "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
+            "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read")
 
 _lib = None
 _lock = threading.Lock()
@@ -62,6 +63,15 @@ def load_library(path: str | None = None):
         lib.rsa_last_device_status.restype = i
         lib.rsa_plan_describe.argtypes = [i, i, i, i, i, i, i, i, sz, ctypes.POINTER(ctypes.c_longlong)]
         lib.rsa_plan_describe.restype = i
+        lib.rsa_profile_enable.argtypes = [i]
+        lib.rsa_profile_enable.restype = i
+        lib.rsa_profile_kinds.argtypes = []
+        lib.rsa_profile_kinds.restype = i
+        lib.rsa_profile_kind_name.argtypes = [i]
+        lib.rsa_profile_kind_name.restype = ctypes.c_char_p
+        lib.rsa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                         ctypes.POINTER(ctypes.c_longlong)]
+        lib.rsa_profile_read.restype = i
         if path is None:
             _lib = lib
         return lib
@@ -103,6 +113,25 @@ def plan_describe(B: int, H: int, L: int, d: int, N: int, causal: bool, dtype: t
 def last_device_status(stream: torch.cuda.Stream | None = None) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(load_library().rsa_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def profile_enable(on: bool) -> None:
+    """Bracket every library kernel launch with CUDA events on its stream (benchmarks)."""
+    rc = load_library().rsa_profile_enable(int(bool(on)))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kernel name: (total ms, launches)} accumulated since the last read; waits for the events."""
+    lib = load_library()
+    n = lib.rsa_profile_kinds()
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    rc = lib.rsa_profile_read(ms, cnt)
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_profile_read")
+    return {lib.rsa_profile_kind_name(k).decode(): (ms[k], cnt[k]) for k in range(n) if cnt[k]}
 
 
 def _check_qkv(*ts):

@@ -44,13 +44,17 @@ def rel_l2(a, b):
     return np.linalg.norm((a - b).ravel()) / (den if den > 0 else 1.0)
 
 
-def check(got, ref, dtype, name):
+def check(got, ref, dtype, name, magnitude_scaled=False):
+    """magnitude_scaled: for the supplementary unscaled-input cases, whose outputs exceed 8 in
+    magnitude (one bf16 ulp is then 0.0625), the max-abs bound is taken relative to the
+    tensor's largest magnitude."""
     err = np.abs(got - ref).max() if got.size else 0.0
     if dtype == "f32":
         assert err <= F32_MAXABS, f"{name}: max-abs {err:.3e} > {F32_MAXABS}"
     else:
         r = rel_l2(got, ref)
-        assert err <= BF16_MAXABS and r <= BF16_RELL2, f"{name}: max-abs {err:.3e}, rel-L2 {r:.3e}"
+        bound = BF16_MAXABS * (max(1.0, float(np.abs(ref).max())) if magnitude_scaled else 1.0)
+        assert err <= bound and r <= BF16_RELL2, f"{name}: max-abs {err:.3e} (bound {bound:.3e}), rel-L2 {r:.3e}"
 
 
 def run(x, N, causal, *, bwd=True, ws_budget=0):
@@ -66,13 +70,14 @@ def run(x, N, causal, *, bwd=True, ws_budget=0):
     return {n: np64(t) for n, t in out.items()}
 
 
-def check_full(orc, x, got, causal, bwd=True):
+def check_full(orc, x, got, causal, bwd=True, magnitude_scaled=False):
     o, lse = orc.forward(x.q, x.k, x.v, causal)
-    check(got["O"], o, x.dtype, "O")
-    np.testing.assert_allclose(got["lse"], lse, rtol=0, atol=1e-5 if x.dtype == "f32" else 1e-3)
+    check(got["O"], o, x.dtype, "O", magnitude_scaled)
+    tol = 1e-5 if x.dtype == "f32" else 1e-3
+    np.testing.assert_allclose(got["lse"], lse, rtol=tol if magnitude_scaled else 0, atol=tol)
     if bwd:
         for name, ref in zip(("dQ", "dK", "dV"), orc.backward(x.q, x.k, x.v, x.do, causal)):
-            check(got[name], ref, x.dtype, name)
+            check(got[name], ref, x.dtype, name, magnitude_scaled)
 
 
 def check_sampled(orc, x, got, causal, heads, rows, keys):
@@ -252,7 +257,7 @@ def test_sharp_attention(orc, kind):
                     q_extra_scale=extra)
     for causal in (False, True):
         got = run(x, 4, causal)
-        check_full(orc, x, got, causal)
+        check_full(orc, x, got, causal, magnitude_scaled=True)
         o, _ = orc.forward(x.q, x.k, x.v, causal)
         assert rel_l2(got["O"], o) <= BF16_RELL2
 
