@@ -83,9 +83,9 @@ def kernel_model(w):
         "slab_softmax": (0, 4 * p + 2 * p + row),               # S read, P bf16 write, lse
         "pv_ring_rows": (2 * p * d, 2 * p + 2 * t),             # P read, V read, O write
         "rowdot": (0, 2 * t + row),
-        "bwd_slab": (4 * p * d, 2 * p + 2 * p + 4 * t + 2 * row),  # P, dS write; Q K dO V read
-        "dkdv_ring_keys": (4 * p * d, 2 * p + 2 * p + 4 * t),   # P, dS read; dO, Q read; dK, dV
-        "dq_ring_rows": (2 * p * d, 2 * p + 2 * t),             # dS read, K read, dQ write
+        # key-major backward: S^T, dP^T, dV, dK GEMMs; dS^T slab write, Q K V dO read, dK dV write
+        "bwd_keys": (8 * p * d, 2 * p + 6 * t + 2 * row),
+        "dq_ring_rows": (2 * p * d, 2 * p + 2 * t),             # dS^T read, K read, dQ write
     }
 
 

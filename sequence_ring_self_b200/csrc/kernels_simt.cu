@@ -122,15 +122,19 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
-// D_i = dO_i . O_i. The flattened [rows][D] arrays are read as 16-byte vectors: vector t holds
-// elements [8t, 8t + 8) (bf16) or [4t, 4t + 4) (fp32), so TPR = D / (elements per vector)
-// consecutive threads share a row and reduce with shuffles. Warps stride in lockstep.
+// Row statistics for the backward pass, in rows padded to Lp (zeros past L):
+//   D[bh][i] = dO_i . O_i  and, if lse2 is given, lse2[bh][i] = lse[bh][i] * log2(e).
+// The flattened [rows][D] inputs are read as 16-byte vectors: vector t holds elements
+// [8t, 8t + 8) (bf16) or [4t, 4t + 4) (fp32), so TPR = D / (elements per vector) consecutive
+// threads share a row and reduce with shuffles. Warps stride in lockstep.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
     rowdot_kernel(const uint4 *__restrict__ dO, const uint4 *__restrict__ O,
-                  float *__restrict__ Dvec, long long rows) {
+                  const float *__restrict__ lse, float *__restrict__ Dp, float *__restrict__ lse2,
+                  long long BH, int L, int Lp) {
     constexpr int EPV = BF16 ? 8 : 4;
     constexpr int TPR = D / EPV;
+    const long long rows = BH * L;
     const long long total = rows * TPR;
     const int lane = threadIdx.x & 31;
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -158,7 +162,24 @@ __global__ void __launch_bounds__(256)
         }
 #pragma unroll
         for (int o = TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (t < total && (lane % TPR) == 0) Dvec[t / TPR] = s;
+        if (t < total && (lane % TPR) == 0) {
+            const long long r = t / TPR;
+            const long long bh = r / L;
+            const long long out = bh * Lp + (r - bh * L);
+            Dp[out] = s;
+            if (lse2) lse2[out] = lse[r] * kLog2e;
+        }
+    }
+    // padding rows [L, Lp) of every head
+    const int pad = Lp - L;
+    if (pad > 0) {
+        for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+             t < BH * pad; t += stride) {
+            const long long bh = t / pad;
+            const long long out = bh * Lp + L + (t - bh * pad);
+            Dp[out] = 0.f;
+            if (lse2) lse2[out] = 0.f;
+        }
     }
 }
 
@@ -317,7 +338,7 @@ __global__ void __launch_bounds__(256)
         const int i = i0 + ty * 4 + u;
         if (i >= a.r0 + a.R) continue;
         const float l = lse[static_cast<size_t>(bh) * a.L + i];
-        const float Di = Dvec[static_cast<size_t>(bh) * a.L + i];
+        const float Di = Dvec[static_cast<size_t>(bh) * a.Lp + i];
         const size_t roff = (static_cast<size_t>(h) * a.R + (i - a.r0)) * a.Lp;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
@@ -424,9 +445,10 @@ cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int 
     return cudaGetLastError();
 }
 
-cudaError_t launch_rowdot(const void *dO, const void *O, float *Dvec, long long rows, int d,
-                          int bf16, cudaStream_t st) {
-    const long long vectors = rows * d / (bf16 ? 8 : 4);
+cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,
+                          float *lse2, long long BH, int L, int Lp, int d, int bf16,
+                          cudaStream_t st) {
+    const long long vectors = BH * L * d / (bf16 ? 8 : 4);
     long long grid = (vectors + 255) / 256;
     if (grid > 148 * 16) grid = 148 * 16;
     if (grid < 1) grid = 1;
@@ -434,11 +456,11 @@ cudaError_t launch_rowdot(const void *dO, const void *O, float *Dvec, long long 
     auto *a = static_cast<const uint4 *>(dO);
     auto *b = static_cast<const uint4 *>(O);
     if (bf16) {
-        if (d == 64) rowdot_kernel<64, true><<<g, 256, 0, st>>>(a, b, Dvec, rows);
-        else rowdot_kernel<128, true><<<g, 256, 0, st>>>(a, b, Dvec, rows);
+        if (d == 64) rowdot_kernel<64, true><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
+        else rowdot_kernel<128, true><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
     } else {
-        if (d == 32) rowdot_kernel<32, false><<<g, 256, 0, st>>>(a, b, Dvec, rows);
-        else rowdot_kernel<64, false><<<g, 256, 0, st>>>(a, b, Dvec, rows);
+        if (d == 32) rowdot_kernel<32, false><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
+        else rowdot_kernel<64, false><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
     }
     return cudaGetLastError();
 }

@@ -81,9 +81,11 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     p.BH = static_cast<long long>(B) * H;
     p.Lp = (L + 63) / 64 * 64;
     p.c = L / N;
-    // forward: fp32 scores with P written in place; backward: P and dS (bf16, or fp32)
-    p.row_bytes = (dt == RSA_F32 && bwd) ? size_t(8) * p.Lp : size_t(4) * p.Lp;
-    const size_t fixed = bwd ? align_up(size_t(p.BH) * L * 4, kAlign) : 0;
+    // forward: fp32 scores with P written in place (4 B per score); backward: the key-major
+    // bf16 dS^T slab (2 B), or fp32 P and dS on the fp32 path (8 B)
+    p.row_bytes = bwd ? (dt == RSA_F32 ? size_t(8) * p.Lp : size_t(2) * p.Lp) : size_t(4) * p.Lp;
+    // backward: padded row statistics D and lse * log2(e), [2][BH][Lp] fp32
+    const size_t fixed = bwd ? align_up(size_t(2) * p.BH * p.Lp * 4, kAlign) : 0;
     const size_t head_bytes = align_up(size_t(L) * p.row_bytes, kAlign);
     const size_t acc_bytes = (bwd && dt == RSA_BF16) ? 2 * align_up(size_t(L) * d * 4, kAlign) : 0;
     if (budget >= fixed + head_bytes) {
@@ -171,7 +173,8 @@ rsa_status_t device_state(DeviceState **out) {
         if (major != 10) return RSA_ERR_UNSUPPORTED;
         if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return RSA_ERR_CUDA;
-        if (rsa::tc_kernels_configure() != cudaSuccess) return RSA_ERR_CUDA;
+        if (rsa::tc_kernels_configure() != cudaSuccess || rsa::bwd_kernels_configure() != cudaSuccess)
+            return RSA_ERR_CUDA;
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, rsa::g_status_word) != cudaSuccess) return RSA_ERR_CUDA;
         s.status = static_cast<int *>(ptr);
@@ -193,13 +196,12 @@ rsa_status_t device_state(DeviceState **out) {
 // ---------------------------------------------------------------- per-kernel timing
 
 enum Kind {
-    K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_SLAB, K_RING_KEYS, K_DQ,
+    K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_DQ,
     K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
-    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_slab", "dkdv_ring_keys",
-    "dq_ring_rows", "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys",
-    "f32_dq_ring_rows"};
+    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_keys", "dq_ring_rows",
+    "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows"};
 
 struct ProfRec {
     int kind;
@@ -254,15 +256,16 @@ rsa_status_t timed(int kind, cudaStream_t s, F &&launch) {
         if (st_ != RSA_OK) return st_;                                           \
     } while (0)
 
-// 3-D tiled tensor map, 128-byte swizzle, zero fill out of bounds.
+// 3-D tiled tensor map (128-byte swizzle unless told otherwise), zero fill out of bounds.
 bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t d0, uint64_t d1,
-           uint64_t d2, uint64_t pitch1, uint64_t pitch2, uint32_t box0, uint32_t box1) {
+           uint64_t d2, uint64_t pitch1, uint64_t pitch2, uint32_t box0, uint32_t box1,
+           CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     cuuint64_t dims[3] = {d0, d1, d2};
     cuuint64_t strides[2] = {pitch1, pitch2};
     cuuint32_t box[3] = {box0, box1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(m, type, 3, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -431,7 +434,7 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         a.nCT = 0;
         a.ntiles = G.nh * a.nRT;
         a.scale = 1.f;
-        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
+        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, 0, a, dev->sms, s));
     }
     return RSA_OK;
 }
@@ -453,11 +456,14 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
     if (st != RSA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    float *Dvec = reinterpret_cast<float *>(ws + p.off_D);
+    // row statistics [2][BH][Lp]: lse * log2(e), then D
+    float *lse2 = reinterpret_cast<float *>(ws + p.off_D);
+    float *Dvec = lse2 + size_t(p.BH) * p.Lp;
     const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
 
-    // D_i = dO_i . O_i
-    RSA_LAUNCH(K_ROWDOT, rsa::launch_rowdot(dO, O, Dvec, p.BH * L, d, dt == RSA_BF16, s));
+    // D_i = dO_i . O_i and lse_i * log2(e), in rows padded to Lp
+    RSA_LAUNCH(K_ROWDOT, rsa::launch_rowdot(dO, O, lse, Dvec, dt == RSA_BF16 ? lse2 : nullptr, p.BH,
+                                            L, p.Lp, d, dt == RSA_BF16, s));
 
     if (dt == RSA_F32) {
         for (long long g = 0; g < p.ngroups; ++g) {
@@ -478,11 +484,12 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
         return RSA_OK;
     }
 
-    CUtensorMap mQk, mKk, mdOk, mVk, mKmn, mdOmn, mQmn;
-    if (!map_input(&mQk, Q, p, 128) || !map_input(&mKk, K, p, 128) ||
-        !map_input(&mdOk, dO, p, 128) || !map_input(&mVk, V, p, 128) ||
-        !map_input(&mKmn, K, p, 64) || !map_input(&mdOmn, dO, p, 64) ||
-        !map_input(&mQmn, Q, p, 64))
+    CUtensorMap mK128, mV128, mQ64, mdO64, mK64, mStat;
+    if (!map_input(&mK128, K, p, 128) || !map_input(&mV128, V, p, 128) ||
+        !map_input(&mQ64, Q, p, 64) || !map_input(&mdO64, dO, p, 64) || !map_input(&mK64, K, p, 64) ||
+        !map3d(&mStat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2,
+               p.Lp, p.BH, 2, uint64_t(p.Lp) * 4, uint64_t(p.Lp) * 4 * p.BH, 64, 1,
+               CU_TENSOR_MAP_SWIZZLE_NONE))
         return RSA_ERR_CUDA;
     float *acc_dK = p.whole ? nullptr : reinterpret_cast<float *>(ws + p.off_acc);
     float *acc_dV = p.whole ? nullptr
@@ -491,35 +498,25 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
     for (long long g = 0; g < p.ngroups; ++g) {
         const Group G = group_of(p, g);
         SlabArgs a = slab_args(p, G, dev->status);
-        const uint64_t pitch = uint64_t(p.Lp) * 2;
-        const size_t region = size_t(G.nh) * G.R * pitch;  // a multiple of 128 bytes
-        uint8_t *Pb = ws;
-        uint8_t *dSb = ws + region;
-        CUtensorMap mPst, mdSst, mPt, mdSt, mdSk;
-        const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-        if (!map3d(&mPst, bf, Pb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 32) ||
-            !map3d(&mdSst, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 32) ||
-            !map3d(&mPt, bf, Pb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 64) ||
-            !map3d(&mdSt, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 64) ||
-            !map3d(&mdSk, bf, dSb, p.Lp, G.R, G.nh, pitch, pitch * G.R, 64, 128))
+        // key-major dS^T slab of the group: [nh][L keys][R queries], rows padded to 64 queries
+        const uint64_t pitch = uint64_t((G.R + 63) / 64 * 64) * 2;
+        CUtensorMap mdSld;
+        if (!map3d(&mdSld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws, G.R, L, G.nh, pitch, pitch * L, 64, 64))
             return RSA_ERR_CUDA;
-        // P = exp(scale Q K^T - lse) and dS = P (dO V^T - D), as bf16 slabs
-        a.nCT = (p.Lp + 127) / 128;
-        a.ntiles = G.nh * a.nRT * a.nCT;
-        RSA_LAUNCH(K_BWD_SLAB, rsa::launch_bwd_slab(mQk, mKk, mdOk, mVk, mPst, mdSst, lse, Dvec, a, dev->sms, s));
-        // dV_m, dK_m gathered from every query chunk (key-major ring)
+        a.dst_pitch = static_cast<int>(pitch / 2);
         if (!p.whole && G.first_of_head) {
             RSA_TRY(cudaMemsetAsync(acc_dK, 0, size_t(L) * d * 4, s));
             RSA_TRY(cudaMemsetAsync(acc_dV, 0, size_t(L) * d * 4, s));
         }
+        // key-major ring: P^T, dP^T -> dS^T (to the slab); dV_m, dK_m over the query chunks
         a.mode = p.whole ? 0 : (G.last_of_head ? 2 : 1);
-        a.nCT = 0;
         a.ntiles = G.nh * ((L + 127) / 128);
-        RSA_LAUNCH(K_RING_KEYS, rsa::launch_ring_keys(mPt, mdOmn, mdSt, mQmn, dK, dV, acc_dK, acc_dV, a, dev->sms, s));
-        // dQ_n = scale * sum_s dS_n[:, block m] K_m
+        RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat, ws, dK, dV,
+                                                    acc_dK, acc_dV, a, dev->sms, s));
+        // dQ_n = scale * sum_s dS_n[:, block m] K_m, reading the key-major slab
         a.mode = 0;
         a.ntiles = G.nh * a.nRT;
-        RSA_LAUNCH(K_DQ, rsa::launch_ring_rows(mdSk, mKmn, dQ, a, dev->sms, s));
+        RSA_LAUNCH(K_DQ, rsa::launch_ring_rows(mdSld, mK64, dQ, 1, a, dev->sms, s));
     }
     return RSA_OK;
 }

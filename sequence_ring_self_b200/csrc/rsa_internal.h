@@ -26,6 +26,7 @@ struct SlabArgs {
     int nCT;     // column tiles per head (kernel-specific width)
     int ntiles;  // tiles in the launch (before causal skipping)
     int mode;    // kernel-specific (see each kernel)
+    int dst_pitch;  // backward: row pitch (elements) of the key-major dS^T slab
     int *status; // device status word
 };
 
@@ -33,26 +34,29 @@ struct SlabArgs {
 // Each returns a cudaError_t of its launch.
 cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mS,
                            const SlabArgs &a, int num_sms, cudaStream_t st);
-cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
+// a_mn = 0: A is the row-major P slab (O = P V); a_mn = 1: A is the key-major dS^T slab.
+cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out, int a_mn,
                              const SlabArgs &a, int num_sms, cudaStream_t st);
-cudaError_t launch_bwd_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mdO,
-                            const CUtensorMap &mV, const CUtensorMap &mP, const CUtensorMap &mdS,
-                            const float *lse, const float *Dvec, const SlabArgs &a, int num_sms,
+// Fused key-major backward: recompute P^T, dP^T -> dS^T (stored to the dS^T slab), and
+// dV = P^T dO, dK = scale dS^T Q accumulated in TMEM over the group's query blocks.
+// mStat: the padded row statistics [2][BH][Lp] fp32 (lse * log2(e), then D), box 64 x 1 x 1.
+cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mQ,
+                            const CUtensorMap &mdO, const CUtensorMap &mStat, void *dSt, void *dK,
+                            void *dV, float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
                             cudaStream_t st);
-cudaError_t launch_ring_keys(const CUtensorMap &mPt, const CUtensorMap &mdO,
-                             const CUtensorMap &mdSt, const CUtensorMap &mQ, void *dK, void *dV,
-                             float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
-                             cudaStream_t st);
 cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
+cudaError_t bwd_kernels_configure();
 
 // ---- CUDA-core kernels (kernels_simt.cu) -----------------------------------------------
 // Row softmax of the group's fp32 slab, in place: P written as bf16 (p_bf16 = 1) into the
 // first half of each fp32 row, or as fp32 over S (p_bf16 = 0). Writes lse.
 cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int p_bf16,
                                 cudaStream_t st);
-// D_i = dO_i . O_i for all rows of all heads (fp32 result).
-cudaError_t launch_rowdot(const void *dO, const void *O, float *Dvec, long long rows, int d,
-                          int bf16, cudaStream_t st);
+// D_i = dO_i . O_i (and lse2 = lse * log2(e) when lse2 != NULL) for all rows of all heads,
+// written in rows padded to Lp with zeros past L.
+cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,
+                          float *lse2, long long BH, int L, int Lp, int d, int bf16,
+                          cudaStream_t st);
 // fp32 path (every step in fp32 FMA).
 cudaError_t launch_f32_qk_slab(const float *Q, const float *K, float *S, const SlabArgs &a,
                                cudaStream_t st);

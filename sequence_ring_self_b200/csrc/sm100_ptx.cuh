@@ -60,14 +60,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep (woken when the phase completes) for up to
+// `hint_ns` before the answer is false, instead of spinning on the issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Wait until the phase with the given parity of `bar` has completed. Returns false (and
 // raises *abort) if the CTA was aborted or the wait ran past kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0u) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((it & 7u) == 0u) {
             if (*abort) return false;
             if (global_timer_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
@@ -206,6 +220,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(2) << 61;
     return d;
+}
+
+// The same descriptor split into a compile-time constant part (LBO, SBO, version, layout) and
+// the start address field, so that issuing threads only add (address >> 4) per MMA. Shared
+// addresses of a CTA are below 2^18, so the 14-bit start field never carries.
+__host__ __device__ constexpr uint64_t sdesc_const(uint32_t lbo, uint32_t sbo) {
+    return (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+
+__device__ __forceinline__ uint64_t sdesc(uint64_t cst, uint32_t saddr) {
+    return cst | static_cast<uint64_t>(saddr >> 4);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 accumulator,
