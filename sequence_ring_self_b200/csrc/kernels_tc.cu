@@ -26,8 +26,11 @@ constexpr int kThreads = 192;
 using namespace tc;
 
 // ======================================================================================
-// qk_slab: S[h][i - r0][j] = scale * Q_i . K_j   (fp32; -inf where j >= L or causal j > i)
+// qk_slab: S[h][i - r0][j] = log2(e) * scale * Q_i . K_j  (fp32 scores in base-2 units;
+// -inf where j >= L or causal j > i), and per row and 128-column half tile the softmax
+// partials (max_j S, sum_j 2^(S - max)) for the streaming softmax.
 // Tile = 128 query rows x 256 keys; K-loop over d in blocks of 64 (one 128-byte swizzle row).
+// 320 threads: producer, MMA, and 8 epilogue warps (2 per TMEM lane quarter, 128 columns each).
 // ======================================================================================
 template <int D>
 struct QkCfg {
@@ -37,7 +40,7 @@ struct QkCfg {
     static constexpr int B_BYTES = BN * 64 * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = 3;
-    static constexpr int EPI_BYTES = 4 * 2 * 4096;  // per epilogue warp: 2 x (32 rows x 128 B)
+    static constexpr int EPI_BYTES = 8 * 2 * 4096;  // per epilogue warp: 2 x (32 rows x 128 B)
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + (int)sizeof(Ctl);
     static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -64,8 +67,17 @@ __device__ __forceinline__ bool qk_decode(const SlabArgs &a, int t, QkTile &tl) 
     return true;
 }
 
+constexpr int kQkThreads = 320;
+
+__device__ __forceinline__ void softmax_combine(float &m, float &l, float m2, float l2) {
+    const float nm = fmaxf(m, m2);
+    if (nm == -INFINITY) return;
+    l = l * fast_exp2(m - nm) + l2 * fast_exp2(m2 - nm);
+    m = nm;
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kQkThreads, 1)
     qk_slab_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                    const __grid_constant__ CUtensorMap mS, const SlabArgs a) {
     using C = QkCfg<D>;
@@ -77,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        init_ctl(ctl, C::STAGES, 4);
+        init_ctl(ctl, C::STAGES, 8);
         prefetch_tmap(&mQ);
         prefetch_tmap(&mK);
         prefetch_tmap(&mS);
@@ -158,8 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        const int ew = warp - 2, q = warp & 3;
+        const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
         uint8_t *ebuf = epi + ew * 8192;
+        const float sl2 = a.scale * kLog2e;
         int acc = 0;
         uint32_t aph = 0;
         for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
@@ -168,27 +181,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&ctl->tfull[acc], aph, &ctl->abort)) break;
             tc_fence_after();
             const int i = tl.i0 + 32 * q + lane;
+            const int i_min = tl.i0 + 32 * q;  // smallest row of this warp
+            float run_m = -INFINITY, run_l = 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < C::BN / 32; ++cc) {
+            for (int cc = 0; cc < 4; ++cc) {
+                const int col = hf * 128 + cc * 32;
                 uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * C::BN + cc * 32, r);
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * C::BN + col, r);
                 tmem_ld_wait();
+                const int j0 = tl.ct * C::BN + col;
+                float v[32];
+                float cm = -INFINITY;
+                if (j0 + 32 <= a.L && (!a.causal || j0 + 31 <= i_min)) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        v[e] = __uint_as_float(r[e]) * sl2;
+                        cm = fmaxf(cm, v[e]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = j0 + e;
+                        const bool live = j < a.L && !(a.causal && j > i);
+                        v[e] = live ? __uint_as_float(r[e]) * sl2 : -INFINITY;
+                        cm = fmaxf(cm, v[e]);
+                    }
+                }
+                if (cm != -INFINITY) {
+                    float cs = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) cs += fast_exp2(v[e] - cm);
+                    softmax_combine(run_m, run_l, cm, cs);
+                }
                 uint8_t *buf = ebuf + (cc & 1) * 4096;
                 if (lane == 0) bulk_wait_read<1>();
                 __syncwarp();
-                const int j0 = tl.ct * C::BN + cc * 32;
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    float v[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = j0 + 4 * e4 + u;
-                        const bool live = j < a.L && !(a.causal && j > i);
-                        v[u] = live ? __uint_as_float(r[4 * e4 + u]) * a.scale : -INFINITY;
-                    }
+                for (int e4 = 0; e4 < 8; ++e4)
                     *reinterpret_cast<float4 *>(buf + sw128_offset(lane, e4)) =
-                        make_float4(v[0], v[1], v[2], v[3]);
-                }
+                        make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
@@ -199,6 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            if (i < a.r0 + a.R)
+                a.stats[(static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat + 2 * tl.ct + hf] =
+                    make_float2(run_m, run_l);
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
         }
@@ -421,9 +455,9 @@ cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const C
                            const SlabArgs &a, int num_sms, cudaStream_t st) {
     const int grid = tc::grid_for(a.ntiles, num_sms);
     if (a.d == 64)
-        qk_slab_kernel<64><<<grid, kThreads, QkCfg<64>::SMEM, st>>>(mQ, mK, mS, a);
+        qk_slab_kernel<64><<<grid, kQkThreads, QkCfg<64>::SMEM, st>>>(mQ, mK, mS, a);
     else
-        qk_slab_kernel<128><<<grid, kThreads, QkCfg<128>::SMEM, st>>>(mQ, mK, mS, a);
+        qk_slab_kernel<128><<<grid, kQkThreads, QkCfg<128>::SMEM, st>>>(mQ, mK, mS, a);
     return cudaGetLastError();
 }
 

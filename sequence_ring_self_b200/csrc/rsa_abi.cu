@@ -84,6 +84,8 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     // forward: fp32 scores with P written in place (4 B per score); backward: the key-major
     // bf16 dS^T slab (2 B), or fp32 P and dS on the fp32 path (8 B)
     p.row_bytes = bwd ? (dt == RSA_F32 ? size_t(8) * p.Lp : size_t(2) * p.Lp) : size_t(4) * p.Lp;
+    // forward (bf16): plus the per-row softmax partials, one float2 per 128 columns
+    if (!bwd && dt == RSA_BF16) p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
     // backward: padded row statistics D and lse * log2(e), [2][BH][Lp] fp32
     const size_t fixed = bwd ? align_up(size_t(2) * p.BH * p.Lp * 4, kAlign) : 0;
     const size_t head_bytes = align_up(size_t(L) * p.row_bytes, kAlign);
@@ -418,6 +420,10 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         const Group G = group_of(p, g);
         SlabArgs a = slab_args(p, G, dev->status);
         const uint64_t pitch = uint64_t(p.Lp) * 4;  // fp32 row; P (bf16) in its first half
+        a.nCT = (p.Lp + 255) / 256;
+        a.nStat = 2 * a.nCT;
+        a.stats = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(slab) +
+                                             align_up(size_t(G.nh) * G.R * pitch, kAlign));
         CUtensorMap mS, mP;
         if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
                    pitch * G.R, 32, 32) ||
@@ -425,11 +431,10 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
                    pitch * G.R, 64, 128))
             return RSA_ERR_CUDA;
         // ring pass 1: score slab
-        a.nCT = (p.Lp + 255) / 256;
         a.ntiles = G.nh * a.nRT * a.nCT;
         RSA_LAUNCH(K_QK_SLAB, rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
-        // row softmax over the full key length
-        RSA_LAUNCH(K_SOFTMAX, rsa::launch_slab_softmax(slab, lse, a, 1, s));
+        // row softmax over the full key length (partials from the slab GEMM, one streaming pass)
+        RSA_LAUNCH(K_SOFTMAX, rsa::launch_slab_softmax_stream(slab, lse, a, s));
         // ring pass 2: O = P V
         a.nCT = 0;
         a.ntiles = G.nh * a.nRT;

@@ -27,6 +27,8 @@ struct SlabArgs {
     int ntiles;  // tiles in the launch (before causal skipping)
     int mode;    // kernel-specific (see each kernel)
     int dst_pitch;  // backward: row pitch (elements) of the key-major dS^T slab
+    int nStat;      // forward: per-row softmax partials (one per 128 key columns)
+    float2 *stats;  // forward: [nh][R][nStat] (max, sum of 2^(s - max)) in base-2 units
     int *status; // device status word
 };
 
@@ -49,9 +51,13 @@ cudaError_t bwd_kernels_configure();
 
 // ---- CUDA-core kernels (kernels_simt.cu) -----------------------------------------------
 // Row softmax of the group's fp32 slab, in place: P written as bf16 (p_bf16 = 1) into the
-// first half of each fp32 row, or as fp32 over S (p_bf16 = 0). Writes lse.
+// first half of each fp32 row, or as fp32 over S (p_bf16 = 0). Writes lse. Natural-unit
+// scores, statistics computed here (the fp32 path).
 cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int p_bf16,
                                 cudaStream_t st);
+// Row softmax of the bf16 path: scores in base-2 units with per-row partials (a.stats) from
+// the slab GEMM; one streaming pass writes bf16 P in place and lse.
+cudaError_t launch_slab_softmax_stream(float *slab, float *lse, const SlabArgs &a, cudaStream_t st);
 // D_i = dO_i . O_i (and lse2 = lse * log2(e) when lse2 != NULL) for all rows of all heads,
 // written in rows padded to Lp with zeros past L.
 cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,

@@ -148,10 +148,13 @@ def _check_qkv(*ts):
 
 
 def _workspace(nbytes: int, device, workspace):
+    """A caller-supplied workspace is used as it is (the library plans for its size and
+    reports RSA_ERR_WORKSPACE if it is below the smallest plan); otherwise one of the size
+    the budget asks for is allocated."""
     if workspace is None:
         return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
-        raise ValueError("workspace too small or not on the device")
+    if not workspace.is_cuda or workspace.device != device:
+        raise ValueError("workspace must be on the tensors' device")
     return workspace
 
 

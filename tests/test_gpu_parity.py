@@ -296,5 +296,6 @@ def test_library_errors_raise():
         rsa.forward(q, q, q, 3)
     small = torch.empty(1024, dtype=torch.uint8, device=dev)
     q2 = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device=dev)
-    with pytest.raises(ValueError):
+    with pytest.raises(rsa.RSAError) as e:
         rsa.forward(q2, q2, q2, 1, workspace=small)
+    assert e.value.code == rsa.RSA_ERR_WORKSPACE
