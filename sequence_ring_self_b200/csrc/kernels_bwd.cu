@@ -6,20 +6,23 @@
 // of 128 keys (K_m, V_m resident in shared memory) and visits the group's query rows in
 // 64-row blocks, starting at the block of its own chunk and wrapping around:
 //
-//   S^T  = K_m Q_n^T,   dP^T = V_m dO_n^T                   (tcgen05, two TMEM accumulators)
+//   S^T  = K_m Q_n^T,   dP^T = V_m dO_n^T                   (tcgen05, TMEM accumulators)
 //   P^T  = exp(scale S^T - lse_n),  dS^T = P^T (dP^T - D_n)   (epilogue warps, fp32 -> bf16)
-//   dV_m += P^T dO_n,   dK_m += scale dS^T Q_n               (tcgen05, A = P^T / dS^T in smem)
+//   dV_m += P^T dO_n,   dK_m += scale dS^T Q_n               (tcgen05, A operand in TMEM)
 //
-// dS^T is also written to the key-major dS^T slab (each thread stores its key row's 64-byte
-// run) for the dQ ring GEMM, which reads it as an MN-major operand. P never leaves the chip: it is recomputed from lse (the
-// forward's fp32 row statistics), in the manner of recomputation in the backward pass.
+// P never leaves the chip: it is recomputed from lse (the forward's fp32 row statistics), in
+// the manner of recomputation in the backward pass. The epilogue writes P^T and dS^T as bf16
+// pairs back into the TMEM columns it has just read S^T and dP^T from, and the dV/dK MMAs take
+// their A operand from there. dS^T also goes to the key-major dS^T slab (plain 16-byte stores,
+// 64 contiguous bytes per key row) for the dQ ring GEMM, which reads it as an MN-major operand.
 //
-// Roles (320 threads): warp 0 lane 0 issues TMA loads (K/V per tile, Q/dO per step);
-// warp 1 owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the epilogue: warp w reads
-// TMEM lanes 32*(w%4)..+31 (keys) and query columns 32*((w-2)/4)..+31 of each step.
-// Pipelining: S^T/dP^T accumulators and the P^T/dS^T operand buffers are double-buffered, and
-// the MMA warp issues step t's S^T/dP^T before step t-1's dV/dK, so the tensor core works on
-// one step while the epilogue works on the previous one.
+// Roles (320 threads): warp 0 lane 0 issues TMA loads (K/V per key tile, Q/dO and the rows'
+// statistics per step); warp 1 owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the
+// epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (keys) and query columns 32*((w-2)/4)..+31.
+// The S^T/dP^T accumulators are double-buffered and the MMA warp issues step t's S^T/dP^T
+// before step t-1's dV/dK, so the tensor core works on one step while the epilogue works on
+// the previous one. MMAs of one thread execute in issue order, so step t's dV/dK MMAs read
+// P^T/dS^T of buffer b before step t+2's S^T/dP^T MMAs overwrite it.
 #include "tc_common.cuh"
 
 namespace rsa {
@@ -32,28 +35,27 @@ constexpr int kEpiWarps = 8;
 
 template <int D>
 struct BkCfg {
-    static constexpr int QB = 64;                       // query rows per step
-    static constexpr int KV_BYTES = 128 * D * 2;        // resident [128 keys][D] tile
-    static constexpr int KV_SLOTS = D == 64 ? 2 : 1;
-    static constexpr int QT_BYTES = QB * D * 2;         // [64 queries][D] tile
-    static constexpr int STAT_OFF = 2 * QT_BYTES;       // then lse*log2(e) [64] and D [64]
-    static constexpr int STAGE_BYTES = 2 * QT_BYTES + 1024;  // Q, dO, row statistics (padded)
-    static constexpr int STAGES = D == 64 ? 4 : 2;
-    static constexpr int PT_BYTES = 128 * QB * 2;       // [128 keys][64 queries] bf16
-    static constexpr int PBUF_BYTES = 2 * PT_BYTES;     // P^T then dS^T
+    static constexpr int QB = 64;                        // query rows per step
+    static constexpr int KV_BYTES = 128 * D * 2;         // resident [128 keys][D] tile
+    static constexpr int KV_SLOTS = 2;
+    static constexpr int QT_BYTES = QB * D * 2;          // [64 queries][D] tile
+    static constexpr int STAT_OFF = 2 * QT_BYTES;        // then lse*log2(e) [64] and D [64]
+    static constexpr int STAGE_BYTES = 2 * QT_BYTES + 1024;
+    static constexpr int STAGES = D == 64 ? 5 : 2;
     static constexpr int OFF_KV = 0;
     static constexpr int OFF_STAGE = OFF_KV + KV_SLOTS * 2 * KV_BYTES;
-    static constexpr int OFF_P = OFF_STAGE + STAGES * STAGE_BYTES;
-    static constexpr int OFF_CTL = OFF_P + 2 * PBUF_BYTES;
+    static constexpr int OFF_CTL = OFF_STAGE + STAGES * STAGE_BYTES;
     static constexpr uint32_t TMEM_COLS = 512;
-    // TMEM columns: S^T[b] at 128 b, dP^T[b] at 128 b + 64, dV at 256, dK at 256 + D
+    // TMEM columns: S^T[b] at 128 b, dP^T[b] at 128 b + 64, dV at 256, dK at 256 + D.
+    // P^T / dS^T of step t (bf16 pairs) overwrite S^T[b] / dP^T[b]: queries 32h..32h+31 of
+    // step t occupy columns 32h .. 32h + 15 of the buffer.
 };
 
 struct BkCtl {
-    uint64_t full[4], empty[4];      // Q/dO stages
+    uint64_t full[8], empty[8];      // Q/dO stages
     uint64_t kvfull[2], kvempty[2];  // resident K/V slots
-    uint64_t sfull[2], sfree[2];     // S^T/dP^T accumulators
-    uint64_t pready[2], pfree[2];    // P^T/dS^T operand buffers
+    uint64_t sfull[2];               // S^T/dP^T of buffer b computed
+    uint64_t pready[2];              // P^T/dS^T of buffer b written to TMEM
     uint64_t accfull, accempty;      // dV/dK accumulators
     uint64_t drain;
     uint32_t tmem_base;
@@ -130,9 +132,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
     bwd_keys_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                     const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mdO,
                     const __grid_constant__ CUtensorMap mStat, __nv_bfloat16 *__restrict__ dSt,
-                    __nv_bfloat16 *__restrict__ dK,
-                    __nv_bfloat16 *__restrict__ dV, float *__restrict__ acc_dK,
-                    float *__restrict__ acc_dV, const SlabArgs a) {
+                    __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV,
+                    float *__restrict__ acc_dK, float *__restrict__ acc_dV, const SlabArgs a) {
     using C = BkCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1024(smem_raw);
@@ -150,9 +151,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->sfull[b], 1);
-            mbar_init(&ctl->sfree[b], kEpiWarps);
             mbar_init(&ctl->pready[b], kEpiWarps);
-            mbar_init(&ctl->pfree[b], 1);
         }
         mbar_init(&ctl->accfull, 1);
         mbar_init(&ctl->accempty, kEpiWarps);
@@ -234,12 +233,12 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             constexpr uint64_t KM = sdesc_const(16, 1024);    // K-major, 128-byte swizzle
             constexpr uint64_t MN = sdesc_const(8192, 1024);  // MN-major, 64-wide blocks 8 KB apart
             const uint32_t id_s = idesc_bf16_f32(128, C::QB, 0, 0);  // S^T, dP^T
-            const uint32_t id_g = idesc_bf16_f32(128, D, 0, 1);      // dV, dK
+            const uint32_t id_g = idesc_bf16_f32(128, D, 0, 1);      // dV, dK (A in TMEM)
             const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + D;
             Pipe p{0, 0}, kv{0, 0};
             uint32_t gstep = 0, acc_ph = 0;
             bool ok = true;
-            // pending dV/dK work of the previous step
+            // dV/dK work of the previous step, issued after the next step's S^T/dP^T
             bool pend = false, pend_first = false;
             int pend_stage = 0;
             uint32_t pend_b = 0, pend_ph = 0;
@@ -247,18 +246,17 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (!mbar_wait(&ctl->pready[pend_b], pend_ph, &ctl->abort)) return false;
                 if (pend_first && !mbar_wait(&ctl->accempty, acc_ph ^ 1u, &ctl->abort)) return false;
                 tc_fence_after();
-                const uint32_t pt = smem_addr(smem + C::OFF_P + pend_b * C::PBUF_BYTES);
                 const uint32_t st = smem_addr(smem + C::OFF_STAGE + pend_stage * C::STAGE_BYTES);
-                const uint64_t d_p = sdesc(KM, pt), d_ds = sdesc(KM, pt + C::PT_BYTES);
                 const uint64_t d_do = sdesc(MN, st + C::QT_BYTES), d_q = sdesc(MN, st);
+                const uint32_t t_p = tmem + 128 * pend_b, t_ds = t_p + 64;
 #pragma unroll
                 for (int k = 0; k < C::QB / 16; ++k) {
                     const uint32_t en = (pend_first && k == 0) ? 0u : 1u;
-                    tc_mma_bf16(t_dv, d_p + 2 * k, d_do + 128 * k, id_g, en);
-                    tc_mma_bf16(t_dk, d_ds + 2 * k, d_q + 128 * k, id_g, en);
+                    const uint32_t col = (k >> 1) * 32 + (k & 1) * 8;  // 16 queries per MMA
+                    tc_mma_bf16_ts(t_dv, t_p + col, d_do + 128 * k, id_g, en);
+                    tc_mma_bf16_ts(t_dk, t_ds + col, d_q + 128 * k, id_g, en);
                 }
                 tc_commit(&ctl->empty[pend_stage]);
-                tc_commit(&ctl->pfree[pend_b]);
                 pend = false;
                 return true;
             };
@@ -269,17 +267,18 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tc_fence_after();
                 const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
                 const uint32_t vs = ks + C::KV_BYTES;
+                const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, vs);
                 for (int s = 0; s < tl.cnt; ++s) {
-                    const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
-                    if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort) ||
-                        !mbar_wait(&ctl->sfree[b], bph ^ 1u, &ctl->abort)) {
+                    const uint32_t b = gstep & 1u;
+                    if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
                         ok = false;
                         break;
                     }
+                    // buffer b was last read by the dV/dK MMAs of step gstep - 2, issued
+                    // before these (in-order execution)
                     tc_fence_after();
                     const uint32_t st = smem_addr(smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES);
                     const uint32_t t_s = tmem + 128 * b, t_p = t_s + 64;
-                    const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, vs);
                     const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb)
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     pend_first = s == 0;
                     pend_stage = p.stage;
                     pend_b = b;
-                    pend_ph = bph;
+                    pend_ph = (gstep >> 1) & 1u;
                     pipe_next(p, C::STAGES);
                     ++gstep;
                 }
@@ -332,27 +331,20 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const int i0 = a.r0 + bk_block(tl, s) * 64;
                 const int ic = i0 + 32 * hf;  // first query column of this warp
                 const int r_end = a.r0 + a.R;
-                if (!warp_wait(&ctl->sfull[b], bph, &ctl->abort)) {
+                if (!warp_wait(&ctl->sfull[b], bph, &ctl->abort) ||
+                    !warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t t_s = tmem + lane_base + 128 * b + 32 * hf;
                 uint32_t rs[32], rd[32];
-                tmem_ld32(tmem + lane_base + 128 * b + 32 * hf, rs);
-                tmem_ld32(tmem + lane_base + 128 * b + 64 + 32 * hf, rd);
+                tmem_ld32(t_s, rs);
+                tmem_ld32(t_s + 64, rd);
                 tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->sfree[b]);
                 const bool masked = (a.causal && ic < tl.j0 + 128) || tl.j0 + 128 > a.L ||
                                     ic + 32 > r_end;
                 // row statistics of this warp's 32 queries, loaded with the step's Q/dO stage
-                // (already complete: the stage fed the S^T/dP^T MMAs; the wait makes the TMA
-                // writes visible to this warp)
-                if (!warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort)) {
-                    ok = false;
-                    break;
-                }
                 const float *stat = reinterpret_cast<const float *>(
                     smem + C::OFF_STAGE + ps.stage * C::STAGE_BYTES + C::STAT_OFF) + 32 * hf;
                 uint32_t wp[16], wd[16];
@@ -360,23 +352,11 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     epi_compute<false>(rs, rd, stat, sl2, 0, 0, 0, 0, 0, wp, wd);
                 else
                     epi_compute<true>(rs, rd, stat, sl2, j, ic, a.L, r_end, a.causal, wp, wd);
-                // operand buffer b: free once the dV/dK MMAs of two steps ago are done and the
-                // dS^T store issued from it then has read it
-                if (!warp_wait(&ctl->pfree[b], bph ^ 1u, &ctl->abort)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *pb = smem + C::OFF_P + b * C::PBUF_BYTES;
-                const int row = 32 * q + lane;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint32_t off = sw128_offset(row, 4 * hf + g);
-                    *reinterpret_cast<uint4 *>(pb + off) =
-                        make_uint4(wp[4 * g], wp[4 * g + 1], wp[4 * g + 2], wp[4 * g + 3]);
-                    *reinterpret_cast<uint4 *>(pb + C::PT_BYTES + off) =
-                        make_uint4(wd[4 * g], wd[4 * g + 1], wd[4 * g + 2], wd[4 * g + 3]);
-                }
-                fence_async_smem();
+                // P^T and dS^T over the columns just read, as the dV/dK MMAs' A operands
+                tmem_st16(t_s, wp);
+                tmem_st16(t_s + 64, wd);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->pready[b]);
                 // dS^T row j, queries [ic, ic + 32) of the key-major slab (64 contiguous bytes)

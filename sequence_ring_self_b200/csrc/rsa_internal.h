@@ -42,6 +42,7 @@ cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void 
 // Fused key-major backward: recompute P^T, dP^T -> dS^T (stored to the dS^T slab), and
 // dV = P^T dO, dK = scale dS^T Q accumulated in TMEM over the group's query blocks.
 // mStat: the padded row statistics [2][BH][Lp] fp32 (lse * log2(e), then D), box 64 x 1 x 1.
+// dSt: the key-major dS^T slab of the group [nh][L][a.dst_pitch] bf16.
 cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mQ,
                             const CUtensorMap &mdO, const CUtensorMap &mStat, void *dSt, void *dK,
                             void *dV, float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
