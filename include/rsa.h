@@ -133,6 +133,33 @@ RSA_API int rsa_profile_kinds(void);
 RSA_API const char *rsa_profile_kind_name(int kind); /* NULL if out of range */
 RSA_API rsa_status_t rsa_profile_read(double *ms, long long *launches);
 
+/* Size of the scratch array rsa_forward_noalloc works in: 32 MiB of device memory per GPU
+ * that loads the library, held until the process exits. */
+#define RSA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * rsa_forward for callers that cannot allocate device memory. No counterpart on the pages:
+ * it exists for callers that may not call cudaMalloc, such as code running under another
+ * runtime that owns the device memory pool, or latency-critical paths where an allocation
+ * could synchronise the device. It computes exactly what rsa_forward computes (same
+ * arguments, same outputs) but takes its workspace from a fixed scratch array of
+ * RSA_NOALLOC_SCRATCH_BYTES inside the library, so the caller passes only inputs and outputs;
+ * the slab is processed in as many groups as that scratch requires. It allocates nothing and
+ * calls no allocating routine.
+ * - Problems whose smallest plan does not fit the scratch (rows longer than about 64,000
+ *   keys) are rejected with RSA_ERR_WORKSPACE before anything is launched.
+ * - The first call on a device looks up the scratch array's device address on that device;
+ *   make that first call before any stream capture on the device.
+ * - Every call on a device uses the same scratch array, and it keeps the last call's
+ *   contents (nothing in it needs to start cleared: each call writes every byte it reads).
+ *   Calls whose work overlaps on the GPU (for example on two streams without ordering
+ *   between them) race on the scratch and give wrong results; order them on one stream or
+ *   with events.
+ */
+RSA_API rsa_status_t rsa_forward_noalloc(const void *Q, const void *K, const void *V, void *O,
+                                         float *lse, int B, int H, int L, int d, int N,
+                                         int causal, rsa_dtype_t dt, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,8 @@ RSA_F32, RSA_BF16 = 0, 1
 
 EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
-            "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read")
+            "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
+            "rsa_forward_noalloc")
 
 _lib = None
 _lock = threading.Lock()
@@ -72,6 +73,8 @@ def load_library(path: str | None = None):
         lib.rsa_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double),
                                          ctypes.POINTER(ctypes.c_longlong)]
         lib.rsa_profile_read.restype = i
+        lib.rsa_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+        lib.rsa_forward_noalloc.restype = i
         if path is None:
             _lib = lib
         return lib
@@ -207,6 +210,25 @@ def backward(q, k, v, o, do, lse, N: int, causal: bool = False, *, ws_budget: in
     if rc != RSA_OK:
         raise RSAError(rc, "rsa_backward")
     return dq, dk, dv
+
+
+def forward_noalloc(q, k, v, N: int, causal: bool = False, *, out=None, lse=None,
+                    stream: torch.cuda.Stream | None = None):
+    """rsa_forward without a caller workspace: the library works in its own fixed scratch
+    array (RSA_NOALLOC_SCRATCH_BYTES per GPU), for callers that may not allocate device
+    memory. Pass `out` and `lse` to allocate nothing here either. Calls on one device share
+    the scratch, so calls that overlap on the GPU must not be issued."""
+    _check_qkv(q, k, v)
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = load_library().rsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d,
+                                            N, int(bool(causal)), _dtype_code(q.dtype),
+                                            ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_forward_noalloc")
+    return o, ls
 
 
 class RingSelfAttention(torch.autograd.Function):
