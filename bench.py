@@ -422,13 +422,57 @@ def run_gpu(args, w):
     return 0
 
 
+def run_sweep(args):
+    """The sweep configuration (B=1, H=16, d=64, bf16; L x N x causal): one JSON line per point
+    with the GPU step time and TFLOP/s (documentation numbers; the contract line is the default
+    workload's)."""
+    import torch
+
+    from sequence_ring_self_b200 import build, rsa
+    from sequence_ring_self_b200.inputs import make_inputs
+
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    Ls = [int(x) for x in args.sweep_L.split(",")]
+    Ns = [int(x) for x in args.sweep_N.split(",")]
+    for causal in (False, True):
+        for L in Ls:
+            for N in Ns:
+                w = dict(B=1, H=16, L=L, d=64, N=N, causal=causal, seed=5)
+                x = make_inputs(1, 16, L, 64, seed=5, dtype="bf16")
+                q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+                o, lse = rsa.forward(q, k, v, N, causal)
+                rsa.backward(q, k, v, o, do, lse, N, causal)
+                torch.cuda.synchronize()
+                times = []
+                for _ in range(args.steps):
+                    flush.zero_()
+                    torch.cuda._sleep(2_000_000)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    o, lse = rsa.forward(q, k, v, N, causal)
+                    rsa.backward(q, k, v, o, do, lse, N, causal)
+                    e1.record()
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1))
+                ms = statistics.median(times)
+                print(json.dumps({"sweep_point": {"L": L, "N": N, "causal": causal}, "ms_per_step": ms,
+                                  "tflops": step_flops(w) / ms / 1e9,
+                                  "tokens_per_s": L / ms * 1e3}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="bert")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["sweep"], default="bert")
+    ap.add_argument("--sweep-L", default="1024,2048,4096,8192,16384,32768")
+    ap.add_argument("--sweep-N", default="1,2,4,8,16")
     ap.add_argument("--ws-budget", type=int, default=0, help="workspace budget in bytes (0: default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU seconds of the oracle sample reported as cpu_baseline")
@@ -440,6 +484,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload == "sweep":
+        return run_sweep(args)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
