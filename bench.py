@@ -293,27 +293,39 @@ def run_gpu(args, w):
     clocks = ClockSampler(local)
     clocks.start()
     K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def timed_steps(n, kernel_events):
+        """n steps, each preceded (outside its events) by the L2 flush and a short GPU spin that
+        keeps the launch queue ahead of the GPU; returns the per-step device times (ms)."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        rsa.profile_enable(kernel_events)
+        for i in range(n):
+            flush.zero_()
+            torch.cuda._sleep(guard_cycles)
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+    # the timed region: K steps, no per-kernel events (kernels overlap their prologues with the
+    # previous kernel's tail through programmatic dependent launch)
     dist.barrier()
     torch.cuda.synchronize()
-    rsa.profile_enable(True)
     t0 = time.perf_counter()
-    for i in range(K):
-        flush.zero_()
-        torch.cuda._sleep(guard_cycles)
-        starts[i].record()
-        step()
-        ends[i].record()
-    torch.cuda.synchronize()
+    step_ms = timed_steps(K, False)
     t1 = time.perf_counter()
     dist.barrier()
-    prof = rsa.profile_read()
-    rsa.profile_enable(False)
     clocks.stop()
     if rsa.last_device_status() != rsa.RSA_OK:
         raise RuntimeError("a kernel reported a timeout")
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    # per-kernel durations: the same steps again with every library kernel bracketed by CUDA
+    # events on its stream (the events themselves add about 5 us per kernel to a step)
+    kp = max(3, min(K, args.profile_steps))
+    prof_step_ms = timed_steps(kp, not args.no_kernel_events)
+    prof = rsa.profile_read()
+    rsa.profile_enable(False)
     total_ms = sum(step_ms)
     slowest_ms = dist.max_over_ranks(total_ms, dev)
     flops = step_flops(w)
@@ -364,6 +376,8 @@ def run_gpu(args, w):
                 ph["achieved_tflops"] = fl / avg_s / 1e12
                 ph["tensor_frac"] = ph["achieved_tflops"] / peaks["bf16_tflops"]
         phases.append(ph)
+    if not phases:
+        phases = [{"kernel": "none (no per-kernel events)"}]
     top = phases[0]
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -405,7 +419,8 @@ def run_gpu(args, w):
         "tokens_per_s": tokens_s,
         "step_ms_median": statistics.median(step_ms),
         "e2e": e2e,
-        "gpu_launches": int(sum(n for _, n in prof.values())),
+        "gpu_launches": int(round(sum(n for _, n in prof.values()) / kp * K)),
+        "profiled_pass": {"steps": kp, "ms_per_step_with_kernel_events": statistics.median(prof_step_ms)},
         "roofline": roofline,
         "phases": phases,
         "clocks": clocks.summary(t0, t1),
@@ -480,6 +495,10 @@ def main():
                     help="seconds the whole --impl reference run should take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--no-kernel-events", action="store_true",
+                    help="skip the per-kernel profiled pass (no phases / roofline)")
+    ap.add_argument("--profile-steps", type=int, default=50,
+                    help="steps of the per-kernel profiled pass that follows the timed region")
     ap.add_argument("--flush-mib", type=int, default=512, help="L2 flush buffer (MiB) written before each step")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -172,6 +172,9 @@ __global__ void __launch_bounds__(kBkThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
+    // everything above (barriers, TMEM, descriptor prefetch) overlaps the previous kernel
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
@@ -448,17 +451,16 @@ cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const 
                             const CUtensorMap &mdO, const CUtensorMap &mStat, void *dSt, void *dK,
                             void *dV, float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
                             cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     const int grid = tc::grid_for(a.ntiles, num_sms);
     auto *k = static_cast<__nv_bfloat16 *>(dK);
     auto *v = static_cast<__nv_bfloat16 *>(dV);
     auto *ds = static_cast<__nv_bfloat16 *>(dSt);
     if (a.d == 64)
-        bwd_keys_kernel<64><<<grid, kBkThreads, bk_smem<64>(), st>>>(mK, mV, mQ, mdO, mStat, ds, k,
-                                                                    v, acc_dK, acc_dV, a);
+        e = launch_pdl(bwd_keys_kernel<64>, dim3(grid), dim3(kBkThreads), bk_smem<64>(), st, mK, mV, mQ, mdO, mStat, ds, k, v, acc_dK, acc_dV, a);
     else
-        bwd_keys_kernel<128><<<grid, kBkThreads, bk_smem<128>(), st>>>(mK, mV, mQ, mdO, mStat, ds,
-                                                                      k, v, acc_dK, acc_dV, a);
-    return cudaGetLastError();
+        e = launch_pdl(bwd_keys_kernel<128>, dim3(grid), dim3(kBkThreads), bk_smem<128>(), st, mK, mV, mQ, mdO, mStat, ds, k, v, acc_dK, acc_dV, a);
+    return e;
 }
 
 }  // namespace rsa

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include "rsa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace rsa {
 namespace {
@@ -41,6 +42,8 @@ template <int EPT, bool P_BF16>
 __global__ void __launch_bounds__(1024)
     slab_softmax_kernel(float *__restrict__ slab, float *__restrict__ lse, const SlabArgs a,
                         int wpr) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red_max[32];
     __shared__ float red_sum[32];
     const int tpr = 32 * wpr;
@@ -143,6 +146,8 @@ __device__ __forceinline__ void combine2(float &m, float &l, float m2, float l2)
 // steps only overwrite scores read by earlier ones, so the in-place write is safe.
 __global__ void __launch_bounds__(256)
     slab_softmax_stream_kernel(float *__restrict__ slab, float *__restrict__ lse, const SlabArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const long long nrows = static_cast<long long>(a.nh) * a.R;
     const long long wstride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
@@ -205,42 +210,57 @@ __global__ void __launch_bounds__(256)
     rowdot_kernel(const uint4 *__restrict__ dO, const uint4 *__restrict__ O,
                   const float *__restrict__ lse, float *__restrict__ Dp, float *__restrict__ lse2,
                   long long BH, int L, int Lp) {
+    pdl_wait();
+    pdl_trigger();
     constexpr int EPV = BF16 ? 8 : 4;
     constexpr int TPR = D / EPV;
+    constexpr int U = 4;  // vectors in flight per thread
     const long long rows = BH * L;
     const long long total = rows * TPR;
     const int lane = threadIdx.x & 31;
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long t0 = static_cast<long long>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
-         t0 < total; t0 += stride) {
-        const long long t = t0 + lane;
-        float s = 0.f;
-        if (t < total) {
-            const uint4 a = dO[t], b = O[t];
-            if (BF16) {
-                const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
-                const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+         t0 < total; t0 += U * stride) {
+        uint4 a[U], b[U];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 u = __bfloat1622float2(x[e]), w = __bfloat1622float2(y[e]);
-                    s = fmaf(u.x, w.x, s);
-                    s = fmaf(u.y, w.y, s);
-                }
+        for (int u = 0; u < U; ++u) {
+            const long long t = t0 + u * stride + lane;
+            if (t < total) {
+                a[u] = dO[t];
+                b[u] = O[t];
             } else {
-                const float *x = reinterpret_cast<const float *>(&a);
-                const float *y = reinterpret_cast<const float *>(&b);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s = fmaf(x[e], y[e], s);
+                a[u] = make_uint4(0, 0, 0, 0);
+                b[u] = a[u];
             }
         }
 #pragma unroll
-        for (int o = TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (t < total && (lane % TPR) == 0) {
-            const long long r = t / TPR;
-            const long long bh = r / L;
-            const long long out = bh * Lp + (r - bh * L);
-            Dp[out] = s;
-            if (lse2) lse2[out] = lse[r] * kLog2e;
+        for (int u = 0; u < U; ++u) {
+            const long long t = t0 + u * stride + lane;
+            float s = 0.f;
+            if (BF16) {
+                const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a[u]);
+                const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 p = __bfloat1622float2(x[e]), w = __bfloat1622float2(y[e]);
+                    s = fmaf(p.x, w.x, s);
+                    s = fmaf(p.y, w.y, s);
+                }
+            } else {
+                const float *x = reinterpret_cast<const float *>(&a[u]);
+                const float *y = reinterpret_cast<const float *>(&b[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s = fmaf(x[e], y[e], s);
+            }
+#pragma unroll
+            for (int o = TPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (t < total && (lane % TPR) == 0) {
+                const long long r = t / TPR;
+                const long long bh = r / L;
+                const long long out = bh * Lp + (r - bh * L);
+                Dp[out] = s;
+                if (lse2) lse2[out] = lse[r] * kLog2e;
+            }
         }
     }
     // padding rows [L, Lp) of every head
@@ -265,6 +285,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
     f32_qk_slab_kernel(const float *__restrict__ Q, const float *__restrict__ K,
                        float *__restrict__ S, const SlabArgs a) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float qs[64][D + 1];
     __shared__ float ks[64][D + 1];
     const int h = blockIdx.z;
@@ -313,6 +335,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
     f32_ring_rows_kernel(const float *__restrict__ A, const float *__restrict__ Bm,
                          float *__restrict__ out, const SlabArgs a) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float as[64][65];
     __shared__ float bs[64][D + 1];
     const int h = blockIdx.y;
@@ -373,6 +397,8 @@ __global__ void __launch_bounds__(256)
                         const float *__restrict__ dO, const float *__restrict__ V,
                         const float *__restrict__ lse, const float *__restrict__ Dvec,
                         float *__restrict__ P, float *__restrict__ dS, const SlabArgs a) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float xs[64][D + 1];
     __shared__ float ys[64][D + 1];
     const int h = blockIdx.z;
@@ -431,6 +457,8 @@ template <int D>
 __global__ void __launch_bounds__(256)
     f32_ring_keys_kernel(const float *__restrict__ A, const float *__restrict__ Bm,
                          float *__restrict__ out, float alpha, int accumulate, const SlabArgs a) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float as[64][65];
     __shared__ float bs[64][D + 1];
     const int h = blockIdx.y;
@@ -496,6 +524,7 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int p_bf16,
                                 cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     const int EPT = a.Lp > 16384 ? 32 : 16;
     int wpr = (a.Lp + 32 * EPT - 1) / (32 * EPT);
     if (wpr > 32) return cudaErrorInvalidValue;
@@ -506,77 +535,82 @@ cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int 
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
     if (EPT == 16) {
         if (p_bf16)
-            slab_softmax_kernel<16, true><<<(unsigned)grid, threads, 0, st>>>(slab, lse, a, wpr);
+            e = launch_pdl(slab_softmax_kernel<16, true>, dim3((unsigned)grid), dim3(threads), 0, st, slab, lse, a, wpr);
         else
-            slab_softmax_kernel<16, false><<<(unsigned)grid, threads, 0, st>>>(slab, lse, a, wpr);
+            e = launch_pdl(slab_softmax_kernel<16, false>, dim3((unsigned)grid), dim3(threads), 0, st, slab, lse, a, wpr);
     } else {
         if (p_bf16)
-            slab_softmax_kernel<32, true><<<(unsigned)grid, threads, 0, st>>>(slab, lse, a, wpr);
+            e = launch_pdl(slab_softmax_kernel<32, true>, dim3((unsigned)grid), dim3(threads), 0, st, slab, lse, a, wpr);
         else
-            slab_softmax_kernel<32, false><<<(unsigned)grid, threads, 0, st>>>(slab, lse, a, wpr);
+            e = launch_pdl(slab_softmax_kernel<32, false>, dim3((unsigned)grid), dim3(threads), 0, st, slab, lse, a, wpr);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_slab_softmax_stream(float *slab, float *lse, const SlabArgs &a, cudaStream_t st) {
     const long long rows = static_cast<long long>(a.nh) * a.R;
     long long grid = (rows + 7) / 8;
     if (grid > 148LL * 32) grid = 148LL * 32;
-    slab_softmax_stream_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(slab, lse, a);
-    return cudaGetLastError();
+    return launch_pdl(slab_softmax_stream_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
+                      slab, lse, a);
 }
 
 cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,
                           float *lse2, long long BH, int L, int Lp, int d, int bf16,
                           cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     const long long vectors = BH * L * d / (bf16 ? 8 : 4);
     long long grid = (vectors + 255) / 256;
-    if (grid > 148 * 16) grid = 148 * 16;
+    if (grid > 148 * 8) grid = 148 * 8;  // a full SM of threads each; up to 4 vectors per thread
     if (grid < 1) grid = 1;
     const unsigned g = static_cast<unsigned>(grid);
     auto *a = static_cast<const uint4 *>(dO);
     auto *b = static_cast<const uint4 *>(O);
     if (bf16) {
-        if (d == 64) rowdot_kernel<64, true><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
-        else rowdot_kernel<128, true><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
+        if (d == 64) e = launch_pdl(rowdot_kernel<64, true>, dim3(g), dim3(256), 0, st, a, b, lse, Dp, lse2, BH, L, Lp);
+        else e = launch_pdl(rowdot_kernel<128, true>, dim3(g), dim3(256), 0, st, a, b, lse, Dp, lse2, BH, L, Lp);
     } else {
-        if (d == 32) rowdot_kernel<32, false><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
-        else rowdot_kernel<64, false><<<g, 256, 0, st>>>(a, b, lse, Dp, lse2, BH, L, Lp);
+        if (d == 32) e = launch_pdl(rowdot_kernel<32, false>, dim3(g), dim3(256), 0, st, a, b, lse, Dp, lse2, BH, L, Lp);
+        else e = launch_pdl(rowdot_kernel<64, false>, dim3(g), dim3(256), 0, st, a, b, lse, Dp, lse2, BH, L, Lp);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_f32_qk_slab(const float *Q, const float *K, float *S, const SlabArgs &a,
                                cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     dim3 grid((a.Lp + 63) / 64, (a.R + 63) / 64, a.nh);
-    if (a.d == 32) f32_qk_slab_kernel<32><<<grid, 256, 0, st>>>(Q, K, S, a);
-    else f32_qk_slab_kernel<64><<<grid, 256, 0, st>>>(Q, K, S, a);
-    return cudaGetLastError();
+    if (a.d == 32) e = launch_pdl(f32_qk_slab_kernel<32>, dim3(grid), dim3(256), 0, st, Q, K, S, a);
+    else e = launch_pdl(f32_qk_slab_kernel<64>, dim3(grid), dim3(256), 0, st, Q, K, S, a);
+    return e;
 }
 
 cudaError_t launch_f32_ring_rows(const float *A, const float *Bm, float *out, const SlabArgs &a,
                                  cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     dim3 grid((a.R + 63) / 64, a.nh);
-    if (a.d == 32) f32_ring_rows_kernel<32><<<grid, 256, 0, st>>>(A, Bm, out, a);
-    else f32_ring_rows_kernel<64><<<grid, 256, 0, st>>>(A, Bm, out, a);
-    return cudaGetLastError();
+    if (a.d == 32) e = launch_pdl(f32_ring_rows_kernel<32>, dim3(grid), dim3(256), 0, st, A, Bm, out, a);
+    else e = launch_pdl(f32_ring_rows_kernel<64>, dim3(grid), dim3(256), 0, st, A, Bm, out, a);
+    return e;
 }
 
 cudaError_t launch_f32_bwd_slab(const float *Q, const float *K, const float *dO, const float *V,
                                 const float *lse, const float *Dvec, float *P, float *dS,
                                 const SlabArgs &a, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     dim3 grid((a.Lp + 63) / 64, (a.R + 63) / 64, a.nh);
-    if (a.d == 32) f32_bwd_slab_kernel<32><<<grid, 256, 0, st>>>(Q, K, dO, V, lse, Dvec, P, dS, a);
-    else f32_bwd_slab_kernel<64><<<grid, 256, 0, st>>>(Q, K, dO, V, lse, Dvec, P, dS, a);
-    return cudaGetLastError();
+    if (a.d == 32) e = launch_pdl(f32_bwd_slab_kernel<32>, dim3(grid), dim3(256), 0, st, Q, K, dO, V, lse, Dvec, P, dS, a);
+    else e = launch_pdl(f32_bwd_slab_kernel<64>, dim3(grid), dim3(256), 0, st, Q, K, dO, V, lse, Dvec, P, dS, a);
+    return e;
 }
 
 cudaError_t launch_f32_ring_keys(const float *A, const float *Bm, float *out, float alpha,
                                  int accumulate, const SlabArgs &a, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     dim3 grid((a.L + 63) / 64, a.nh);
-    if (a.d == 32) f32_ring_keys_kernel<32><<<grid, 256, 0, st>>>(A, Bm, out, alpha, accumulate, a);
-    else f32_ring_keys_kernel<64><<<grid, 256, 0, st>>>(A, Bm, out, alpha, accumulate, a);
-    return cudaGetLastError();
+    if (a.d == 32) e = launch_pdl(f32_ring_keys_kernel<32>, dim3(grid), dim3(256), 0, st, A, Bm, out, alpha, accumulate, a);
+    else e = launch_pdl(f32_ring_keys_kernel<64>, dim3(grid), dim3(256), 0, st, A, Bm, out, alpha, accumulate, a);
+    return e;
 }
 
 }  // namespace rsa

@@ -102,6 +102,9 @@ __global__ void __launch_bounds__(kQkThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
+    // everything above (barriers, TMEM, descriptor prefetch) overlaps the previous kernel
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -306,6 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
+    // everything above (barriers, TMEM, descriptor prefetch) overlaps the previous kernel
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -453,27 +459,29 @@ cudaError_t tc_kernels_configure() {
 
 cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mS,
                            const SlabArgs &a, int num_sms, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     const int grid = tc::grid_for(a.ntiles, num_sms);
     if (a.d == 64)
-        qk_slab_kernel<64><<<grid, kQkThreads, QkCfg<64>::SMEM, st>>>(mQ, mK, mS, a);
+        e = launch_pdl(qk_slab_kernel<64>, dim3(grid), dim3(kQkThreads), QkCfg<64>::SMEM, st, mQ, mK, mS, a);
     else
-        qk_slab_kernel<128><<<grid, kQkThreads, QkCfg<128>::SMEM, st>>>(mQ, mK, mS, a);
-    return cudaGetLastError();
+        e = launch_pdl(qk_slab_kernel<128>, dim3(grid), dim3(kQkThreads), QkCfg<128>::SMEM, st, mQ, mK, mS, a);
+    return e;
 }
 
 cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out, int a_mn,
                              const SlabArgs &a, int num_sms, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
     const int grid = tc::grid_for(a.ntiles, num_sms);
     auto *o = static_cast<__nv_bfloat16 *>(out);
     if (a.d == 64 && !a_mn)
-        ring_rows_kernel<64, false><<<grid, kThreads, RowsCfg<64>::SMEM, st>>>(mA, mB, o, a);
+        e = launch_pdl(ring_rows_kernel<64, false>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM, st, mA, mB, o, a);
     else if (a.d == 64)
-        ring_rows_kernel<64, true><<<grid, kThreads, RowsCfg<64>::SMEM, st>>>(mA, mB, o, a);
+        e = launch_pdl(ring_rows_kernel<64, true>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM, st, mA, mB, o, a);
     else if (!a_mn)
-        ring_rows_kernel<128, false><<<grid, kThreads, RowsCfg<128>::SMEM, st>>>(mA, mB, o, a);
+        e = launch_pdl(ring_rows_kernel<128, false>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st, mA, mB, o, a);
     else
-        ring_rows_kernel<128, true><<<grid, kThreads, RowsCfg<128>::SMEM, st>>>(mA, mB, o, a);
-    return cudaGetLastError();
+        e = launch_pdl(ring_rows_kernel<128, true>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st, mA, mB, o, a);
+    return e;
 }
 
 }  // namespace rsa

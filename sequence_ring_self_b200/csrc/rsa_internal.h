@@ -8,6 +8,25 @@
 
 namespace rsa {
 
+// Launch with programmatic stream serialisation: the kernel may start (and run its prologue)
+// while the previous kernel in the stream finishes; it calls pdl_wait() before touching memory
+// the previous kernel writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // One group of the slab schedule: heads [bh0, bh0 + nh) and, inside each of them, the query
 // rows [r0, r0 + R). The group's score slab lives in the workspace as [nh][R][Lp].
 struct Group {

@@ -230,6 +230,16 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ dependent launches
+
+// Programmatic dependent launch: wait until the grid this one depends on (the previous kernel
+// in the stream) has completed and its memory is visible; then let the next grid start its
+// prologue. Both are no-ops for a grid launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile (sm_100 format:
