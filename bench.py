@@ -83,9 +83,12 @@ def kernel_model(w):
         "slab_softmax": (0, 4 * p + 2 * p + row),               # S read, P bf16 write, lse
         "pv_ring_rows": (2 * p * d, 2 * p + 2 * t),             # P read, V read, O write
         "rowdot": (0, 2 * t + row),
-        # key-major backward: S^T, dP^T, dV, dK GEMMs; dS^T slab write, Q K V dO read, dK dV write
-        "bwd_keys": (8 * p * d, 2 * p + 6 * t + 2 * row),
-        "dq_ring_rows": (2 * p * d, 2 * p + 2 * t),             # dS^T read, K read, dQ write
+        # key-major backward: dP^T, dV, dK (+ the recomputed S^T, not counted); Q K V dO read,
+        # dK dV write, the rows' lse and D read
+        "bwd_keys": (6 * p * d, 6 * t + 2 * row),
+        # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO K V read, dQ
+        # write, lse and D read
+        "bwd_rows": (2 * p * d, 5 * t + 2 * row),
     }
 
 

@@ -67,8 +67,10 @@ typedef enum { RSA_F32 = 0, RSA_BF16 = 1 } rsa_dtype_t;
  * range of rows (a multiple of 128) of one head. `budget_bytes` caps the workspace: the
  * returned size is that of the largest plan that fits the budget (or of the smallest plan if
  * none fits). budget_bytes == 0 asks for the default plan (at most 1 GiB).
- * for_backward selects the backward call's needs (it also keeps per-row D_i and, for
- * row-range groups, fp32 dK/dV accumulators).
+ * for_backward selects the backward call's needs: on the bf16 path the backward keeps no
+ * slab (every score tile is recomputed on the chip) and needs only the padded per-row
+ * statistics, 8 * B * H * roundup(L, 64) bytes, whatever the budget; the fp32 path keeps fp32
+ * P and dS slabs, grouped as above, plus the same statistics.
  * Returns 0 if the arguments are invalid or unsupported.
  */
 RSA_API size_t rsa_workspace_size(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt,
@@ -90,7 +92,8 @@ RSA_API rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, vo
  * Backward pass on the same ring schedule: recomputes P from Q, K and lse, forms
  * dP = dO V^T and dS = P * (dP - D) with D_i = dO_i . O_i, then
  * dV_m = sum_n P_n[:, block m]^T dO_n, dK_m = scale sum_n dS_n[:, block m]^T Q_n and
- * dQ_n = scale sum_s dS_n[:, block m] K_m.
+ * dQ_n = scale sum_s dS_n[:, block m] K_m. On the bf16 path the key-major sums (dV, dK) and
+ * the query-major sum (dQ) run as two kernels that each recompute the score tiles they need.
  * In:  Q, K, V, O, dO [B,H,L,d] device dtype dt; lse [B,H,L] fp32 from rsa_forward.
  * Out: dQ, dK, dV [B,H,L,d] device dtype dt.
  * workspace: device, >= rsa_workspace_size(..., for_backward = 1, ...), 256-byte aligned.

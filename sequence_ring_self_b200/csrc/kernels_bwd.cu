@@ -13,8 +13,8 @@
 // P never leaves the chip: it is recomputed from lse (the forward's fp32 row statistics), in
 // the manner of recomputation in the backward pass. The epilogue writes P^T and dS^T as bf16
 // pairs back into the TMEM columns it has just read S^T and dP^T from, and the dV/dK MMAs take
-// their A operand from there. dS^T also goes to the key-major dS^T slab (plain 16-byte stores,
-// 64 contiguous bytes per key row) for the dQ ring GEMM, which reads it as an MN-major operand.
+// their A operand from there. dQ comes from the row-major companion kernel below, which
+// recomputes S, P, dP and dS for its query rows, so no dS slab is ever written.
 //
 // Roles (320 threads): warp 0 lane 0 issues TMA loads (K/V per key tile, Q/dO and the rows'
 // statistics per step); warp 1 owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the
@@ -42,9 +42,11 @@ struct BkCfg {
     static constexpr int STAT_OFF = 2 * QT_BYTES;        // then lse*log2(e) [64] and D [64]
     static constexpr int STAGE_BYTES = 2 * QT_BYTES + 1024;
     static constexpr int STAGES = D == 64 ? 5 : 2;
+    static constexpr int OUT_BUFS = D == 64 ? 2 : 1;     // 2 KB staging buffers per warp
     static constexpr int OFF_KV = 0;
     static constexpr int OFF_STAGE = OFF_KV + KV_SLOTS * 2 * KV_BYTES;
-    static constexpr int OFF_CTL = OFF_STAGE + STAGES * STAGE_BYTES;
+    static constexpr int OFF_OUT = OFF_STAGE + STAGES * STAGE_BYTES;
+    static constexpr int OFF_CTL = OFF_OUT + kEpiWarps * OUT_BUFS * 2048;
     static constexpr uint32_t TMEM_COLS = 512;
     // TMEM columns: S^T[b] at 128 b, dP^T[b] at 128 b + 64, dV at 256, dK at 256 + D.
     // P^T / dS^T of step t (bf16 pairs) overwrite S^T[b] / dP^T[b]: queries 32h..32h+31 of
@@ -123,6 +125,12 @@ __device__ __forceinline__ void epi_compute(const uint32_t (&rs)[32], const uint
     }
 }
 
+// 16-byte chunk g of row r in a [32 rows][64 bytes] staging tile, 64-byte swizzle (the
+// chunk index is XORed with bits 7..8 of the row's byte offset).
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t g) {
+    return row * 64u + ((g ^ ((row >> 1) & 3u)) << 4);
+}
+
 __device__ __forceinline__ int bk_block(const BkTile &tl, int s) {
     return tl.lo + ring_block(tl.first, s, tl.cnt);
 }
@@ -131,9 +139,8 @@ template <int D>
 __global__ void __launch_bounds__(kBkThreads, 1)
     bwd_keys_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                     const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mdO,
-                    const __grid_constant__ CUtensorMap mStat, __nv_bfloat16 *__restrict__ dSt,
-                    __nv_bfloat16 *__restrict__ dK, __nv_bfloat16 *__restrict__ dV,
-                    float *__restrict__ acc_dK, float *__restrict__ acc_dV, const SlabArgs a) {
+                    const __grid_constant__ CUtensorMap mStat, const __grid_constant__ CUtensorMap mdK,
+                    const __grid_constant__ CUtensorMap mdV, const SlabArgs a) {
     using C = BkCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1024(smem_raw);
@@ -163,6 +170,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         prefetch_tmap(&mQ);
         prefetch_tmap(&mdO);
         prefetch_tmap(&mStat);
+        prefetch_tmap(&mdK);
+        prefetch_tmap(&mdV);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
@@ -321,6 +330,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
         const float sl2 = a.scale * kLog2e;
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
+        int obuf = 0;
         uint32_t gstep = 0, acc_ph = 0;
         Pipe ps{0, 0};  // the Q/dO stage of the current step (same order as the producer's)
         bool ok = true;
@@ -362,63 +373,45 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->pready[b]);
-                // dS^T row j, queries [ic, ic + 32) of the key-major slab (64 contiguous bytes)
-                if (j < a.L) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(
-                        dSt + (static_cast<size_t>(tl.h) * a.L + j) * a.dst_pitch + (ic - a.r0));
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_uint4(wd[4 * g], wd[4 * g + 1], wd[4 * g + 2], wd[4 * g + 3]);
-                }
                 ++gstep;
                 pipe_next(ps, C::STAGES);
             }
             if (!ok) break;
-            // dV_m and dK_m of this key tile
+            // dV_m and dK_m of this key tile (scale dS^T Q for dK), bf16 through the staging
+            // buffer: warp (q, hf) stores keys j0 + 32q .. +31, columns hf*D/2 .. +D/2
             if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
             tc_fence_after();
-            const bool key_ok = j < a.L;
-            const size_t orow = (static_cast<size_t>(bh) * a.L + (key_ok ? j : 0)) * D;
-            const size_t arow = static_cast<size_t>(key_ok ? j : 0) * D;  // one head per group
+            const int jw = tl.j0 + 32 * q;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
                 const float mul = which ? a.scale : 1.f;
-                __nv_bfloat16 *o = which ? dK : dV;
-                float *accp = which ? acc_dK : acc_dV;
 #pragma unroll 1
                 for (int cc = 0; cc < D / 64; ++cc) {
                     const int col = hf * (D / 2) + cc * 32;
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_base + 256 + which * D + col, r);
                     tmem_ld_wait();
-                    if (!key_ok) continue;
-                    float v[32];
+                    if (jw >= a.L) continue;  // the whole 32-row box lies past the sequence
+                    uint8_t *buf = obase + obuf * 2048;
+                    obuf = obuf + 1 == C::OUT_BUFS ? 0 : obuf + 1;
+                    if (lane == 0) bulk_wait_read<C::OUT_BUFS - 1>();
+                    __syncwarp();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]) * mul;
-                    if (a.mode != 0) {
-                        float4 *ap = reinterpret_cast<float4 *>(accp + arow + col);
+                    for (int g = 0; g < 4; ++g) {
+                        uint32_t w[4];
 #pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            const float4 x = ap[g];
-                            v[4 * g] += x.x;
-                            v[4 * g + 1] += x.y;
-                            v[4 * g + 2] += x.z;
-                            v[4 * g + 3] += x.w;
-                        }
-                        if (a.mode == 1) {
-#pragma unroll
-                            for (int g = 0; g < 8; ++g)
-                                ap[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-                            continue;
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            w[u] = pack_bf16x2(__uint_as_float(r[8 * g + 2 * u]) * mul,
+                                               __uint_as_float(r[8 * g + 2 * u + 1]) * mul);
+                        *reinterpret_cast<uint4 *>(buf + sw64_offset(lane, g)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    uint4 *op = reinterpret_cast<uint4 *>(o + orow + col);
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        op[g] = make_uint4(pack_bf16x2(v[8 * g], v[8 * g + 1]),
-                                           pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
-                                           pack_bf16x2(v[8 * g + 4], v[8 * g + 5]),
-                                           pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_3d(which ? &mdK : &mdV, buf, col, jw, bh);
+                        bulk_commit();
+                    }
                 }
             }
             tc_fence_before();
@@ -426,6 +419,437 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             if (lane == 0) mbar_arrive(&ctl->accempty);
             acc_ph ^= 1u;
         }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && ctl->abort) atomicExch(a.status, 5);
+}
+
+
+// ====================================================================== dQ on the query ring
+//
+// The row-major half of the backward pass. Seen from query chunk n the ring brings key
+// chunk m = (n + s) mod N at step s; this kernel takes that view for a tile of 128 queries
+// (Q_n, dO_n and their row statistics resident in shared memory) and visits the keys in
+// blocks of KN keys, starting at the block of its own chunk and wrapping around:
+//
+//   S  = Q_n K_m^T,   dP = dO_n V_m^T                       (tcgen05, TMEM accumulators)
+//   dS = exp(scale S - lse_n) (dP - D_n)                     (epilogue warps, fp32 -> bf16)
+//   dQ_n += scale dS K_m                                      (tcgen05, A operand in TMEM)
+//
+// S and dP are recomputed instead of read back from the key-major kernel: the extra MMA work
+// costs less than a dS slab round trip through HBM. Each thread of the epilogue owns one query
+// row, so its statistics lse_i and D_i are two registers.
+//
+// Roles (320 threads) as in the key-major kernel: warp 0 lane 0 issues TMA loads, warp 1
+// owns TMEM and lane 0 issues tcgen05.mma, warps 2..9 are the epilogue (TMEM lanes
+// 32*(w%4)..+31 are its query rows; it takes keys KN/2*((w-2)/4) .. +KN/2 of each block).
+// S is double-buffered, dP single-buffered: the epilogue loads dP first and releases it
+// (dpfree) before it works on S, so the next block's dP MMAs wait only for that load.
+// Each poll of a barrier by the MMA thread stalls the tensor pipe for about a hundred cycles,
+// so blocks are as wide as TMEM allows (KN = 128 keys for d = 64). Q and dO are copied into
+// TMEM once per unit (tcgen05.cp) and the S and dP MMAs take them from there: with both
+// operands in shared memory a 128 x 128 x 16 MMA reads 8 KB per 64 cycles, all the shared
+// memory bandwidth there is, and the K/V loads of later blocks would slow it down.
+// dQ leaves TMEM through a per-warp swizzled staging buffer and TMA stores.
+
+constexpr int kBrThreads = 320;
+
+template <int D>
+struct BrCfg {
+    static constexpr int KN = D == 64 ? 128 : 64;        // keys per step
+    static constexpr int QT_BYTES = 128 * D * 2;         // [128 queries][D] tile
+    static constexpr int STAT_OFF = 2 * QT_BYTES;        // lse*log2(e) [128], then D [128]
+    static constexpr int SLOT_BYTES = 2 * QT_BYTES + 1024;
+    static constexpr int Q_SLOTS = 2;
+    static constexpr int KB_BYTES = KN * D * 2;          // [KN keys][D] block
+    static constexpr int KCHUNK = KN * 128;              // one 64-column box of a block
+    static constexpr int STAGE_BYTES = 2 * KB_BYTES;     // K block, V block
+    static constexpr int STAGES = D == 64 ? 3 : 2;
+    static constexpr int OUT_BUFS = D == 64 ? 2 : 1;     // 2 KB staging buffers per warp
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_STAGE = OFF_Q + Q_SLOTS * SLOT_BYTES;
+    static constexpr int OFF_OUT = OFF_STAGE + STAGES * STAGE_BYTES;
+    static constexpr int OFF_CTL = OFF_OUT + kEpiWarps * OUT_BUFS * 2048;
+    static constexpr uint32_t TMEM_COLS = 512;
+    // TMEM columns: S[b] at KN b, dP at 2 KN, dQ at 3 KN, then the unit's Q and dO as bf16
+    // pairs (the A operands of the S and dP MMAs, D / 2 columns each). dS of a step (bf16
+    // pairs) overwrites S[b]: keys 32g .. 32g + 31 of the block occupy columns 32g .. 32g + 15.
+    static constexpr uint32_t T_DP = 2 * KN, T_DQ = 3 * KN, T_Q = T_DQ + D, T_DO = T_Q + D / 2;
+    static_assert(T_DO + D / 2 <= TMEM_COLS, "TMEM columns");
+};
+
+struct BrCtl {
+    uint64_t full[8], empty[8];    // K/V block stages
+    uint64_t qfull[2], qempty[2];  // resident Q/dO/statistics slots
+    uint64_t sfull[2];             // S[b] and dP computed
+    uint64_t dpfree;               // dP loaded by every epilogue warp
+    uint64_t pready[2];            // dS of buffer b written to TMEM
+    uint64_t accfull, accempty;    // dQ accumulator
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int D>
+constexpr int br_smem() {
+    return 1024 + BrCfg<D>::OFF_CTL + static_cast<int>(sizeof(BrCtl));
+}
+
+struct BrTile {
+    int h, i0, cnt, first;
+};
+
+// Work unit t = (128-query tile, head), longest causal tiles (largest queries) first. The
+// key blocks (kn keys each) the tile can see are 0 .. cnt - 1; the ring starts at the block
+// holding the first key of the tile's own chunk.
+__device__ __forceinline__ void br_decode(const SlabArgs &a, int t, int kn, BrTile &tl) {
+    const int u = t / a.nh;
+    tl.h = t - u * a.nh;
+    const int nqt = (a.L + 127) / 128;
+    const int qt = a.causal ? nqt - 1 - u : u;
+    tl.i0 = qt * 128;
+    const int end = a.causal ? min(a.L, tl.i0 + 128) : a.L;
+    tl.cnt = (end + kn - 1) / kn;
+    const int n = tl.i0 / a.c;
+    tl.first = min((n * a.c) / kn, tl.cnt - 1);
+}
+
+// dS = 2^(S * scale * log2(e) - lse * log2(e)) (dP - D) for 32 keys of one query row, packed
+// to bf16 pairs. MASK zeroes keys j >= L and (causal) j > i.
+template <bool MASK>
+__device__ __forceinline__ void br_compute(const uint32_t (&rs)[32], const uint32_t *rd, float sl2,
+                                           float lse2, float Di, int j0, int i, int L, int causal,
+                                           uint32_t (&wd)[16]) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float v[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float p = fast_exp2(fmaf(__uint_as_float(rs[e + u]), sl2, -lse2));
+            if (MASK) {
+                const int j = j0 + e + u;
+                p = (j >= L || (causal && j > i)) ? 0.f : p;
+            }
+            v[u] = p * (__uint_as_float(rd[e + u]) - Di);
+        }
+        wd[e >> 1] = pack_bf16x2(v[0], v[1]);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBrThreads, 1)
+    bwd_rows_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mdO,
+                    const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                    const __grid_constant__ CUtensorMap mStat,
+                    const __grid_constant__ CUtensorMap mdQ, const SlabArgs a) {
+    using C = BrCfg<D>;
+    constexpr int KN = C::KN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align_1024(smem_raw);
+    BrCtl *ctl = reinterpret_cast<BrCtl *>(smem + C::OFF_CTL);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int s = 0; s < C::Q_SLOTS; ++s) {
+            mbar_init(&ctl->qfull[s], 1);
+            // released by the copies of Q and dO into TMEM and by every epilogue warp once
+            // it holds the rows' statistics in registers
+            mbar_init(&ctl->qempty[s], 1 + kEpiWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->sfull[b], 1);
+            mbar_init(&ctl->pready[b], kEpiWarps);
+        }
+        mbar_init(&ctl->dpfree, kEpiWarps);
+        mbar_init(&ctl->accfull, 1);
+        mbar_init(&ctl->accempty, kEpiWarps);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&mQ);
+        prefetch_tmap(&mdO);
+        prefetch_tmap(&mK);
+        prefetch_tmap(&mV);
+        prefetch_tmap(&mStat);
+        prefetch_tmap(&mdQ);
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            Pipe p{0, 0}, qs{0, 0};
+            bool issued[C::STAGES], qissued[C::Q_SLOTS];
+            uint32_t ipar[C::STAGES], qpar[C::Q_SLOTS];
+            for (int s = 0; s < C::STAGES; ++s) issued[s] = false, ipar[s] = 0;
+            for (int s = 0; s < C::Q_SLOTS; ++s) qissued[s] = false, qpar[s] = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
+                BrTile tl;
+                br_decode(a, t, KN, tl);
+                const int bh = a.bh0 + tl.h;
+                if (!mbar_wait(&ctl->qempty[qs.stage], qs.phase ^ 1u, &ctl->abort)) break;
+                {
+                    uint8_t *slot = smem + C::OFF_Q + qs.stage * C::SLOT_BYTES;
+                    uint64_t *bar = &ctl->qfull[qs.stage];
+                    mbar_arrive_expect_tx(bar, 2 * C::QT_BYTES + 1024);
+#pragma unroll
+                    for (int kb = 0; kb < D / 64; ++kb) {
+                        tma_load_3d(slot + kb * 16384, &mQ, bar, kb * 64, tl.i0, bh);
+                        tma_load_3d(slot + C::QT_BYTES + kb * 16384, &mdO, bar, kb * 64, tl.i0, bh);
+                    }
+                    tma_load_3d(slot + C::STAT_OFF, &mStat, bar, tl.i0, bh, 0);        // lse * log2(e)
+                    tma_load_3d(slot + C::STAT_OFF + 512, &mStat, bar, tl.i0, bh, 1);  // D
+                    qissued[qs.stage] = true;
+                    qpar[qs.stage] = qs.phase;
+                    pipe_next(qs, C::Q_SLOTS);
+                }
+                for (int s = 0; s < tl.cnt; ++s) {
+                    const int j0 = ring_block(tl.first, s, tl.cnt) * KN;
+                    if (!mbar_wait(&ctl->empty[p.stage], p.phase ^ 1u, &ctl->abort)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES;
+                    uint64_t *bar = &ctl->full[p.stage];
+                    mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+#pragma unroll
+                    for (int kb = 0; kb < D / 64; ++kb) {
+                        tma_load_3d(st + kb * C::KCHUNK, &mK, bar, kb * 64, j0, bh);
+                        tma_load_3d(st + C::KB_BYTES + kb * C::KCHUNK, &mV, bar, kb * 64, j0, bh);
+                    }
+                    issued[p.stage] = true;
+                    ipar[p.stage] = p.phase;
+                    pipe_next(p, C::STAGES);
+                }
+            }
+            for (int s = 0; s < C::STAGES; ++s)
+                if (issued[s]) drain_wait(&ctl->full[s], ipar[s]);
+            for (int s = 0; s < C::Q_SLOTS; ++s)
+                if (qissued[s]) drain_wait(&ctl->qfull[s], qpar[s]);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint64_t KM = sdesc_const(16, 1024);          // K-major, 128-byte swizzle
+            constexpr uint64_t MN = sdesc_const(C::KCHUNK, 1024);   // MN-major, 64-wide boxes
+            const uint32_t id_s = idesc_bf16_f32(128, KN, 0, 0);    // S, dP
+            const uint32_t id_g = idesc_bf16_f32(128, D, 0, 1);     // dQ (A in TMEM)
+            const uint32_t t_dp = tmem + C::T_DP, t_dq = tmem + C::T_DQ;
+            Pipe p{0, 0}, qs{0, 0};
+            uint32_t gstep = 0, acc_ph = 0;
+            bool ok = true;
+            bool pend = false, pend_first = false;
+            int pend_stage = 0;
+            uint32_t pend_b = 0, pend_ph = 0;
+            auto grad = [&](void) -> bool {
+                if (!mbar_wait(&ctl->pready[pend_b], pend_ph, &ctl->abort)) return false;
+                if (pend_first && !mbar_wait(&ctl->accempty, acc_ph ^ 1u, &ctl->abort)) return false;
+                tc_fence_after();
+                const uint32_t st = smem_addr(smem + C::OFF_STAGE + pend_stage * C::STAGE_BYTES);
+                const uint64_t d_k = sdesc(MN, st);
+                const uint32_t t_ds = tmem + KN * pend_b;
+#pragma unroll
+                for (int k = 0; k < KN / 16; ++k) {
+                    const uint32_t en = (pend_first && k == 0) ? 0u : 1u;
+                    const uint32_t col = (k >> 1) * 32 + (k & 1) * 8;  // 16 keys per MMA
+                    tc_mma_bf16_ts(t_dq, t_ds + col, d_k + 128 * k, id_g, en);
+                }
+                tc_commit(&ctl->empty[pend_stage]);
+                pend = false;
+                return true;
+            };
+            for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
+                BrTile tl;
+                br_decode(a, t, KN, tl);
+                if (!mbar_wait(&ctl->qfull[qs.stage], qs.phase, &ctl->abort)) break;
+                tc_fence_after();
+                {
+                    // Q, dO -> TMEM (after the previous unit's S/dP MMAs, in issue order)
+                    const uint32_t slot = smem_addr(smem + C::OFF_Q + qs.stage * C::SLOT_BYTES);
+                    const uint64_t d_q = sdesc(KM, slot), d_do = sdesc(KM, slot + C::QT_BYTES);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t o = (k >> 2) * 1024 + 2 * (k & 3);
+                        tc_cp_128x256b(tmem + C::T_Q + 8 * k, d_q + o);
+                        tc_cp_128x256b(tmem + C::T_DO + 8 * k, d_do + o);
+                    }
+                    tc_commit(&ctl->qempty[qs.stage]);
+                }
+                for (int s = 0; s < tl.cnt; ++s) {
+                    const uint32_t b = gstep & 1u;
+                    if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = smem_addr(smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES);
+                    const uint32_t t_s = tmem + KN * b;
+                    const uint64_t d_k = sdesc(KM, st), d_v = sdesc(KM, st + C::KB_BYTES);
+                    // S[b]: its last reader was the dQ MMAs of step gstep - 2, issued earlier
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * (C::KCHUNK >> 4) + 2 * (k & 3);
+                        tc_mma_bf16_ts(t_s, tmem + C::T_Q + 8 * k, d_k + ko, id_s, k ? 1u : 0u);
+                    }
+                    // dP: every epilogue warp has loaded the previous step's dP
+                    if (gstep > 0 && !mbar_wait(&ctl->dpfree, (gstep - 1) & 1u, &ctl->abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * (C::KCHUNK >> 4) + 2 * (k & 3);
+                        tc_mma_bf16_ts(t_dp, tmem + C::T_DO + 8 * k, d_v + ko, id_s, k ? 1u : 0u);
+                    }
+                    tc_commit(&ctl->sfull[b]);
+                    if (pend && !grad()) {
+                        ok = false;
+                        break;
+                    }
+                    pend = true;
+                    pend_first = s == 0;
+                    pend_stage = p.stage;
+                    pend_b = b;
+                    pend_ph = (gstep >> 1) & 1u;
+                    pipe_next(p, C::STAGES);
+                    ++gstep;
+                }
+                if (!ok) break;
+                if (pend && !grad()) break;
+                tc_commit(&ctl->accfull);
+                acc_ph ^= 1u;
+                pipe_next(qs, C::Q_SLOTS);
+            }
+            tc_commit(&ctl->drain);
+            drain_wait(&ctl->drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        constexpr int NCH = KN / 64;  // 32-key chunks per warp and step
+        const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
+        const float sl2 = a.scale * kLog2e;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
+        uint32_t gstep = 0, acc_ph = 0;
+        int obuf = 0;
+        Pipe qs{0, 0};
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
+            BrTile tl;
+            br_decode(a, t, KN, tl);
+            const int bh = a.bh0 + tl.h;
+            const int iw = tl.i0 + 32 * q;  // this warp's first query row
+            const int i = iw + lane;         // this thread's query row
+            if (!warp_wait(&ctl->qfull[qs.stage], qs.phase, &ctl->abort)) break;
+            const float *stat = reinterpret_cast<const float *>(
+                smem + C::OFF_Q + qs.stage * C::SLOT_BYTES + C::STAT_OFF);
+            const float lse2 = stat[32 * q + lane], Di = stat[128 + 32 * q + lane];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->qempty[qs.stage]);
+            pipe_next(qs, C::Q_SLOTS);
+            for (int s = 0; s < tl.cnt; ++s) {
+                const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
+                const int jw = ring_block(tl.first, s, tl.cnt) * KN + hf * (KN / 2);  // first key
+                if (!warp_wait(&ctl->sfull[b], bph, &ctl->abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t t_s = tmem + lane_base + KN * b + hf * (KN / 2);
+                uint32_t rd[NCH][32], rs[32];
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) tmem_ld32(tmem + lane_base + C::T_DP + hf * (KN / 2) + 32 * c, rd[c]);
+                tmem_ld32(t_s, rs);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->dpfree);
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    if (c > 0) {
+                        tmem_ld32(t_s + 32 * c, rs);
+                        tmem_ld_wait();
+                    }
+                    const int jc = jw + 32 * c;
+                    uint32_t wd[16];
+                    if (jc + 32 <= a.L && !(a.causal && jc + 31 > iw))
+                        br_compute<false>(rs, rd[c], sl2, lse2, Di, 0, 0, 0, 0, wd);
+                    else
+                        br_compute<true>(rs, rd[c], sl2, lse2, Di, jc, i, a.L, a.causal, wd);
+                    // dS over the S columns just read, as the dQ MMAs' A operand
+                    tmem_st16(t_s + 32 * c, wd);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->pready[b]);
+                ++gstep;
+            }
+            if (!ok) break;
+            // dQ of this query tile: scale * accumulator, bf16, through the staging buffer
+            if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
+            acc_ph ^= 1u;
+            tc_fence_after();
+            uint32_t r[D / 64][32];
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc)
+                tmem_ld32(tmem + lane_base + C::T_DQ + hf * (D / 2) + 32 * cc, r[cc]);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->accempty);
+            if (iw >= a.L) continue;  // the whole 32-row box lies past the sequence
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                uint8_t *buf = obase + obuf * 2048;
+                obuf = obuf + 1 == C::OUT_BUFS ? 0 : obuf + 1;
+                if (lane == 0) bulk_wait_read<C::OUT_BUFS - 1>();
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        w[u] = pack_bf16x2(__uint_as_float(r[cc][8 * g + 2 * u]) * a.scale,
+                                           __uint_as_float(r[cc][8 * g + 2 * u + 1]) * a.scale);
+                    *reinterpret_cast<uint4 *>(buf + sw64_offset(lane, g)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&mdQ, buf, hf * (D / 2) + 32 * cc, iw, bh);
+                    bulk_commit();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -440,27 +864,36 @@ __global__ void __launch_bounds__(kBkThreads, 1)
 }  // namespace
 
 cudaError_t bwd_kernels_configure() {
-    cudaError_t e = cudaFuncSetAttribute(bwd_keys_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bk_smem<64>());
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(bwd_keys_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                bk_smem<128>());
+    const cudaFuncAttribute smem = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(bwd_keys_kernel<64>, smem, bk_smem<64>());
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_keys_kernel<128>, smem, bk_smem<128>());
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_rows_kernel<64>, smem, br_smem<64>());
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_rows_kernel<128>, smem, br_smem<128>());
+    return e;
 }
 
 cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mQ,
-                            const CUtensorMap &mdO, const CUtensorMap &mStat, void *dSt, void *dK,
-                            void *dV, float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
-                            cudaStream_t st) {
-    cudaError_t e = cudaSuccess;
+                            const CUtensorMap &mdO, const CUtensorMap &mStat,
+                            const CUtensorMap &mdK, const CUtensorMap &mdV, const SlabArgs &a,
+                            int num_sms, cudaStream_t st) {
     const int grid = tc::grid_for(a.ntiles, num_sms);
-    auto *k = static_cast<__nv_bfloat16 *>(dK);
-    auto *v = static_cast<__nv_bfloat16 *>(dV);
-    auto *ds = static_cast<__nv_bfloat16 *>(dSt);
     if (a.d == 64)
-        e = launch_pdl(bwd_keys_kernel<64>, dim3(grid), dim3(kBkThreads), bk_smem<64>(), st, mK, mV, mQ, mdO, mStat, ds, k, v, acc_dK, acc_dV, a);
-    else
-        e = launch_pdl(bwd_keys_kernel<128>, dim3(grid), dim3(kBkThreads), bk_smem<128>(), st, mK, mV, mQ, mdO, mStat, ds, k, v, acc_dK, acc_dV, a);
-    return e;
+        return launch_pdl(bwd_keys_kernel<64>, dim3(grid), dim3(kBkThreads), bk_smem<64>(), st,
+                          mK, mV, mQ, mdO, mStat, mdK, mdV, a);
+    return launch_pdl(bwd_keys_kernel<128>, dim3(grid), dim3(kBkThreads), bk_smem<128>(), st, mK,
+                      mV, mQ, mdO, mStat, mdK, mdV, a);
+}
+
+cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mK,
+                            const CUtensorMap &mV, const CUtensorMap &mStat,
+                            const CUtensorMap &mdQ, const SlabArgs &a, int num_sms,
+                            cudaStream_t st) {
+    const int grid = tc::grid_for(a.ntiles, num_sms);
+    if (a.d == 64)
+        return launch_pdl(bwd_rows_kernel<64>, dim3(grid), dim3(kBrThreads), br_smem<64>(), st,
+                          mQ, mdO, mK, mV, mStat, mdQ, a);
+    return launch_pdl(bwd_rows_kernel<128>, dim3(grid), dim3(kBrThreads), br_smem<128>(), st, mQ,
+                      mdO, mK, mV, mStat, mdQ, a);
 }
 
 }  // namespace rsa

@@ -253,12 +253,10 @@ __global__ void __launch_bounds__(kQkThreads, 1)
 }
 
 // ======================================================================================
-// ring_rows: out[bh][i][:] = scale * sum_j A(i, j) * B[bh][j][:]   (bf16 out)
-// A is a bf16 slab: either row-major P[h][i - r0][j], read K-major in 128 x 64 boxes
-// (A_MN = false, ring pass 2: O = P V), or the key-major dS^T[h][j][i - r0], read MN-major in
-// two 64 x 64 boxes (A_MN = true, dQ = scale dS K). B ([L][D], V or K) is the MN-major
-// operand, read in 64-row boxes 64 columns wide. K-loop over 64-key blocks in ring order
-// starting at the tile's own chunk; causal tiles stop at their diagonal block.
+// ring_rows: out[bh][i][:] = scale * sum_j P(i, j) * V[bh][j][:]   (bf16 out; ring pass 2)
+// P is the row-major bf16 slab P[h][i - r0][j], read K-major in 128 x 64 boxes. V ([L][D])
+// is the MN-major operand, read in 64-row boxes 64 columns wide. K-loop over 64-key blocks
+// in ring order starting at the tile's own chunk; causal tiles stop at their diagonal block.
 // ======================================================================================
 template <int D>
 struct RowsCfg {
@@ -285,7 +283,7 @@ __device__ __forceinline__ void rows_decode(const SlabArgs &a, int t, RowsTile &
     tl.first = min((n * a.c) / 64, tl.nkb - 1);
 }
 
-template <int D, bool A_MN>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     ring_rows_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                      __nv_bfloat16 *__restrict__ out, const SlabArgs a) {
@@ -332,12 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *sa = stages + p.stage * C::STAGE_BYTES;
                     uint64_t *bar = &ctl->full[p.stage];
                     mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                    if (A_MN) {
-                        tma_load_3d(sa, &mA, bar, tl.i0 - a.r0, kb * 64, tl.h);
-                        tma_load_3d(sa + 8192, &mA, bar, tl.i0 - a.r0 + 64, kb * 64, tl.h);
-                    } else {
-                        tma_load_3d(sa, &mA, bar, kb * 64, tl.i0 - a.r0, tl.h);
-                    }
+                    tma_load_3d(sa, &mA, bar, kb * 64, tl.i0 - a.r0, tl.h);
 #pragma unroll
                     for (int dp = 0; dp < D / 64; ++dp)
                         tma_load_3d(sa + C::A_BYTES + dp * 8192, &mB, bar, dp * 64, kb * 64,
@@ -356,10 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             Pipe p{0, 0};
             int acc = 0;
             uint32_t aph = 0;
-            const uint32_t idesc = idesc_bf16_f32(128, D, A_MN ? 1 : 0, 1);
-            constexpr uint64_t DA = A_MN ? sdesc_const(8192, 1024) : sdesc_const(16, 1024);
-            constexpr uint64_t DB = sdesc_const(8192, 1024);
-            constexpr uint32_t KSTEP_A = A_MN ? 128 : 2;  // 16 K-elements in 16-byte units
+            const uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint64_t DA = sdesc_const(16, 1024);    // K-major P
+            constexpr uint64_t DB = sdesc_const(8192, 1024);  // MN-major V
+            constexpr uint32_t KSTEP_A = 2;  // 16 K-elements in 16-byte units
             bool ok = true;
             for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
                 RowsTile tl;
@@ -449,10 +442,8 @@ cudaError_t tc_kernels_configure() {
     if (e != cudaSuccess) return e;
     RSA_SMEM(qk_slab_kernel<64>, QkCfg<64>::SMEM)
     RSA_SMEM(qk_slab_kernel<128>, QkCfg<128>::SMEM)
-    RSA_SMEM((ring_rows_kernel<64, false>), RowsCfg<64>::SMEM)
-    RSA_SMEM((ring_rows_kernel<128, false>), RowsCfg<128>::SMEM)
-    RSA_SMEM((ring_rows_kernel<64, true>), RowsCfg<64>::SMEM)
-    RSA_SMEM((ring_rows_kernel<128, true>), RowsCfg<128>::SMEM)
+    RSA_SMEM(ring_rows_kernel<64>, RowsCfg<64>::SMEM)
+    RSA_SMEM(ring_rows_kernel<128>, RowsCfg<128>::SMEM)
 #undef RSA_SMEM
     return cudaSuccess;
 }
@@ -468,20 +459,15 @@ cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const C
     return e;
 }
 
-cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out, int a_mn,
+cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
                              const SlabArgs &a, int num_sms, cudaStream_t st) {
-    cudaError_t e = cudaSuccess;
     const int grid = tc::grid_for(a.ntiles, num_sms);
     auto *o = static_cast<__nv_bfloat16 *>(out);
-    if (a.d == 64 && !a_mn)
-        e = launch_pdl(ring_rows_kernel<64, false>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM, st, mA, mB, o, a);
-    else if (a.d == 64)
-        e = launch_pdl(ring_rows_kernel<64, true>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM, st, mA, mB, o, a);
-    else if (!a_mn)
-        e = launch_pdl(ring_rows_kernel<128, false>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st, mA, mB, o, a);
-    else
-        e = launch_pdl(ring_rows_kernel<128, true>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st, mA, mB, o, a);
-    return e;
+    if (a.d == 64)
+        return launch_pdl(ring_rows_kernel<64>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM,
+                          st, mA, mB, o, a);
+    return launch_pdl(ring_rows_kernel<128>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st,
+                      mA, mB, o, a);
 }
 
 }  // namespace rsa

@@ -43,7 +43,7 @@ struct Plan {
     long long ngroups;
     size_t row_bytes;   // slab bytes per row (all slabs of the pass)
     size_t slab_bytes;  // slab region
-    size_t off_D, off_acc, total;
+    size_t off_D, total;
 };
 
 bool args_ok(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *why) {
@@ -81,15 +81,26 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     p.BH = static_cast<long long>(B) * H;
     p.Lp = (L + 63) / 64 * 64;
     p.c = L / N;
-    // forward: fp32 scores with P written in place (4 B per score); backward: the key-major
-    // bf16 dS^T slab (2 B), or fp32 P and dS on the fp32 path (8 B)
-    p.row_bytes = bwd ? (dt == RSA_F32 ? size_t(8) * p.Lp : size_t(2) * p.Lp) : size_t(4) * p.Lp;
-    // forward (bf16): plus the per-row softmax partials, one float2 per 128 columns
-    if (!bwd && dt == RSA_BF16) p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
     // backward: padded row statistics D and lse * log2(e), [2][BH][Lp] fp32
     const size_t fixed = bwd ? align_up(size_t(2) * p.BH * p.Lp * 4, kAlign) : 0;
+    if (bwd && dt == RSA_BF16) {
+        // the bf16 backward recomputes every score tile on the chip: no slab, one group
+        p.whole = 1;
+        p.Gh = p.BH;
+        p.R = L;
+        p.ngroups = 1;
+        p.row_bytes = 0;
+        p.slab_bytes = 0;
+        p.off_D = 0;
+        p.total = fixed;
+        return p;
+    }
+    // forward: fp32 scores with P written in place (4 B per score); backward (fp32 path):
+    // fp32 P and dS (8 B)
+    p.row_bytes = bwd ? size_t(8) * p.Lp : size_t(4) * p.Lp;
+    // forward (bf16): plus the per-row softmax partials, one float2 per 128 columns
+    if (!bwd && dt == RSA_BF16) p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
     const size_t head_bytes = align_up(size_t(L) * p.row_bytes, kAlign);
-    const size_t acc_bytes = (bwd && dt == RSA_BF16) ? 2 * align_up(size_t(L) * d * 4, kAlign) : 0;
     if (budget >= fixed + head_bytes) {
         p.whole = 1;
         long long gh = static_cast<long long>((budget - fixed) / head_bytes);
@@ -98,12 +109,11 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
         p.ngroups = (p.BH + p.Gh - 1) / p.Gh;
         p.slab_bytes = align_up(size_t(p.Gh) * L * p.row_bytes, kAlign);
         p.off_D = p.slab_bytes;
-        p.off_acc = p.off_D + fixed;
-        p.total = p.off_acc;
+        p.total = p.off_D + fixed;
     } else {
         p.whole = 0;
         p.Gh = 1;
-        size_t avail = budget > fixed + acc_bytes ? budget - fixed - acc_bytes : 0;
+        size_t avail = budget > fixed ? budget - fixed : 0;
         long long r = static_cast<long long>(avail / p.row_bytes) / 128 * 128;
         if (r < 128) r = 128;
         if (r >= L) r = L;  // only when L <= 128: a whole head is the minimum plan
@@ -113,8 +123,7 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
             p.ngroups = p.BH;
             p.slab_bytes = head_bytes;
             p.off_D = p.slab_bytes;
-            p.off_acc = p.off_D + fixed;
-            p.total = p.off_acc;
+            p.total = p.off_D + fixed;
             return p;
         }
         p.R = static_cast<int>(r);
@@ -122,8 +131,7 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
         p.ngroups = p.BH * per_head;
         p.slab_bytes = align_up(size_t(p.R) * p.row_bytes, kAlign);
         p.off_D = p.slab_bytes;
-        p.off_acc = p.off_D + fixed;
-        p.total = p.off_acc + acc_bytes;
+        p.total = p.off_D + fixed;
     }
     return p;
 }
@@ -198,11 +206,11 @@ rsa_status_t device_state(DeviceState **out) {
 // ---------------------------------------------------------------- per-kernel timing
 
 enum Kind {
-    K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_DQ,
+    K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_BWD_ROWS,
     K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
-    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_keys", "dq_ring_rows",
+    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_keys", "bwd_rows",
     "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows"};
 
 struct ProfRec {
@@ -276,6 +284,12 @@ bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t 
 bool map_input(CUtensorMap *m, const void *base, const Plan &p, uint32_t rows) {
     return map3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, p.d, p.L, p.BH, uint64_t(p.d) * 2,
                  uint64_t(p.L) * p.d * 2, 64, rows);
+}
+
+// Output tensor [BH][L][d] bf16 written by TMA stores of 32 x 32 boxes (64-byte swizzle).
+bool map_output(CUtensorMap *m, void *base, const Plan &p) {
+    return map3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, p.d, p.L, p.BH, uint64_t(p.d) * 2,
+                 uint64_t(p.L) * p.d * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -439,7 +453,7 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         a.nCT = 0;
         a.ntiles = G.nh * a.nRT;
         a.scale = 1.f;
-        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, 0, a, dev->sms, s));
+        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
     }
     return RSA_OK;
 }
@@ -489,40 +503,35 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
         return RSA_OK;
     }
 
-    CUtensorMap mK128, mV128, mQ64, mdO64, mK64, mStat;
+    // Two kernels over the whole problem (one group): the key-major ring gives dK and dV,
+    // the query-major ring gives dQ; both recompute S and dP tile by tile from Q, K, V, dO
+    // and the row statistics, so nothing but the statistics goes through HBM.
+    CUtensorMap mK128, mV128, mQ64, mdO64, mStat64, mQ128, mdO128, mK64, mV64, mStat128;
+    CUtensorMap mdQ, mdK, mdV;
+    const uint64_t stat_pitch = uint64_t(p.Lp) * 4;
     if (!map_input(&mK128, K, p, 128) || !map_input(&mV128, V, p, 128) ||
-        !map_input(&mQ64, Q, p, 64) || !map_input(&mdO64, dO, p, 64) || !map_input(&mK64, K, p, 64) ||
-        !map3d(&mStat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2,
-               p.Lp, p.BH, 2, uint64_t(p.Lp) * 4, uint64_t(p.Lp) * 4 * p.BH, 64, 1,
-               CU_TENSOR_MAP_SWIZZLE_NONE))
+        !map_input(&mQ64, Q, p, 64) || !map_input(&mdO64, dO, p, 64) ||
+        !map_input(&mQ128, Q, p, 128) || !map_input(&mdO128, dO, p, 128) ||
+        !map_input(&mK64, K, p, 64) || !map_input(&mV64, V, p, 64) ||
+        !map3d(&mStat64, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2, p.Lp, p.BH, 2, stat_pitch,
+               stat_pitch * p.BH, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !map3d(&mStat128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2, p.Lp, p.BH, 2, stat_pitch,
+               stat_pitch * p.BH, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !map_output(&mdQ, dQ, p) || !map_output(&mdK, dK, p) || !map_output(&mdV, dV, p))
         return RSA_ERR_CUDA;
-    float *acc_dK = p.whole ? nullptr : reinterpret_cast<float *>(ws + p.off_acc);
-    float *acc_dV = p.whole ? nullptr
-                            : reinterpret_cast<float *>(ws + p.off_acc +
-                                                        align_up(size_t(L) * d * 4, kAlign));
-    for (long long g = 0; g < p.ngroups; ++g) {
-        const Group G = group_of(p, g);
-        SlabArgs a = slab_args(p, G, dev->status);
-        // key-major dS^T slab of the group: [nh][L keys][R queries], rows padded to 64 queries
-        const uint64_t pitch = uint64_t((G.R + 63) / 64 * 64) * 2;
-        CUtensorMap mdSld;
-        if (!map3d(&mdSld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws, G.R, L, G.nh, pitch, pitch * L, 64, 64))
-            return RSA_ERR_CUDA;
-        a.dst_pitch = static_cast<int>(pitch / 2);
-        if (!p.whole && G.first_of_head) {
-            RSA_TRY(cudaMemsetAsync(acc_dK, 0, size_t(L) * d * 4, s));
-            RSA_TRY(cudaMemsetAsync(acc_dV, 0, size_t(L) * d * 4, s));
-        }
-        // key-major ring: P^T, dP^T -> dS^T (to the slab); dV_m, dK_m over the query chunks
-        a.mode = p.whole ? 0 : (G.last_of_head ? 2 : 1);
-        a.ntiles = G.nh * ((L + 127) / 128);
-        RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat, ws, dK, dV,
-                                                    acc_dK, acc_dV, a, dev->sms, s));
-        // dQ_n = scale * sum_s dS_n[:, block m] K_m, reading the key-major slab
-        a.mode = 0;
-        a.ntiles = G.nh * a.nRT;
-        RSA_LAUNCH(K_DQ, rsa::launch_ring_rows(mdSld, mK64, dQ, 1, a, dev->sms, s));
-    }
+    const Group G = group_of(p, 0);
+    SlabArgs a = slab_args(p, G, dev->status);
+    // key-major ring: P^T, dP^T -> dS^T in TMEM; dV_m, dK_m over all query blocks
+    a.mode = 0;
+    a.ntiles = G.nh * ((L + 127) / 128);
+    RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat64, mdK, mdV, a,
+                                                dev->sms, s));
+    // query-major ring: S, dP -> dS in TMEM; dQ_n = scale * sum_m dS_nm K_m
+    a.ntiles = G.nh * ((L + 127) / 128);
+    // (blocks of 128 keys for d = 64, of 64 keys for d = 128)
+    const CUtensorMap &mKr = d == 64 ? mK128 : mK64, &mVr = d == 64 ? mV128 : mV64;
+    RSA_LAUNCH(K_BWD_ROWS, rsa::launch_bwd_rows(mQ128, mdO128, mKr, mVr, mStat128, mdQ, a,
+                                                dev->sms, s));
     return RSA_OK;
 }
 

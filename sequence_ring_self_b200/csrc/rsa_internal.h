@@ -45,7 +45,6 @@ struct SlabArgs {
     int nCT;     // column tiles per head (kernel-specific width)
     int ntiles;  // tiles in the launch (before causal skipping)
     int mode;    // kernel-specific (see each kernel)
-    int dst_pitch;  // backward: row pitch (elements) of the key-major dS^T slab
     int nStat;      // forward: per-row softmax partials (one per 128 key columns)
     float2 *stats;  // forward: [nh][R][nStat] (max, sum of 2^(s - max)) in base-2 units
     int *status; // device status word
@@ -55,16 +54,24 @@ struct SlabArgs {
 // Each returns a cudaError_t of its launch.
 cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mS,
                            const SlabArgs &a, int num_sms, cudaStream_t st);
-// a_mn = 0: A is the row-major P slab (O = P V); a_mn = 1: A is the key-major dS^T slab.
-cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out, int a_mn,
+// O = P V from the row-major bf16 P slab (mA, 128 x 64 boxes) and V (mB, 64 x 64 boxes).
+cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
                              const SlabArgs &a, int num_sms, cudaStream_t st);
-// Fused key-major backward: recompute P^T, dP^T -> dS^T (stored to the dS^T slab), and
-// dV = P^T dO, dK = scale dS^T Q accumulated in TMEM over the group's query blocks.
+// Key-major backward: recompute P^T, dP^T -> dS^T in TMEM, and dV = P^T dO, dK = scale dS^T Q
+// accumulated in TMEM over the group's query blocks.
 // mStat: the padded row statistics [2][BH][Lp] fp32 (lse * log2(e), then D), box 64 x 1 x 1.
-// dSt: the key-major dS^T slab of the group [nh][L][a.dst_pitch] bf16.
+// mdK/mdV: [BH][L][d] bf16, 32 x 32 boxes, 64-byte swizzle (store).
 cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mQ,
-                            const CUtensorMap &mdO, const CUtensorMap &mStat, void *dSt, void *dK,
-                            void *dV, float *acc_dK, float *acc_dV, const SlabArgs &a, int num_sms,
+                            const CUtensorMap &mdO, const CUtensorMap &mStat,
+                            const CUtensorMap &mdK, const CUtensorMap &mdV, const SlabArgs &a,
+                            int num_sms, cudaStream_t st);
+// Row-major backward: recompute S, dP -> dS in TMEM per 128-query tile and dQ = scale dS K.
+// mQ/mdO: 64 x 128 boxes; mK/mV: 64 x 128 boxes for d = 64, 64 x 64 for d = 128 (the key
+// block of a step); mStat: as above with 128 x 1 x 1 boxes;
+// mdQ: [BH][L][d] bf16, 32 x 32 boxes, 64-byte swizzle (store).
+cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mK,
+                            const CUtensorMap &mV, const CUtensorMap &mStat,
+                            const CUtensorMap &mdQ, const SlabArgs &a, int num_sms,
                             cudaStream_t st);
 cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
 cudaError_t bwd_kernels_configure();

@@ -196,6 +196,14 @@ __device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem,
         : "memory");
 }
 
+// Asynchronous copy of a 128-row x 32-byte matrix from shared memory (described by a matrix
+// descriptor, as an MMA operand would be) into TMEM: row r goes to lane r, 8 columns from
+// taddr. Executes in issue order with this thread's tcgen05.mma, so an MMA issued after it
+// sees the copied data; tcgen05.commit tracks its completion.
+__device__ __forceinline__ void tc_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Each thread of the warp writes its TMEM lane, 16 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(

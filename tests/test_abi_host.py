@@ -62,7 +62,7 @@ def test_argument_errors_are_reported_before_any_launch(lib, call):
     assert call(lib, dt=7) == rsa.RSA_ERR_UNSUPPORTED
     assert call(lib, ptr=0) == rsa.RSA_ERR_INVALID_ARG               # null
     assert call(lib, ptr=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG        # misaligned
-    assert call(lib, ws_bytes=1024) == rsa.RSA_ERR_WORKSPACE         # too small
+    assert call(lib, ws_bytes=64) == rsa.RSA_ERR_WORKSPACE           # too small
     assert call(lib, ws=FAKE + 64) == rsa.RSA_ERR_INVALID_ARG        # workspace not 256-aligned
     assert call(lib, ws=0) == rsa.RSA_ERR_INVALID_ARG
 
@@ -81,6 +81,17 @@ def test_workspace_size_invalid_is_zero(lib):
 def test_plans_fit_their_budget_and_grow_with_it(lib, dtype, bwd):
     d = 64
     B, H, L, N = 2, 3, 1000, 8
+    if bwd and dtype == torch.bfloat16:
+        # no slab: one group of every head, the padded row statistics only, for any budget
+        stats = 2 * B * H * 1024 * 4
+        for budget in [1, 1 << 20, 1 << 30, 0]:
+            n = rsa.workspace_size(B, H, L, d, N, False, dtype, bwd, budget)
+            assert n == stats
+            info = rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, n)
+            assert info["fits"] and info["groups"] == 1 and info["rows_per_group"] == L
+            assert info["heads_per_group"] == B * H
+        assert rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, stats - 1)["fits"] is False
+        return
     sizes = []
     for budget in [1, 1 << 18, 1 << 20, 1 << 22, 1 << 24, 1 << 26, 1 << 30]:
         n = rsa.workspace_size(B, H, L, d, N, False, dtype, bwd, budget)

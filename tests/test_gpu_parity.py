@@ -157,12 +157,12 @@ def test_config3_gpt_causal(orc):
 
 
 def test_config4_long_sequence(orc):
-    """B=1 H=16 L=16384 d=128 N=16 bf16, slab groups in sequence (1 GiB default workspace):
-    sampled rows of two heads and sampled keys of one head."""
+    """B=1 H=16 L=16384 d=128 N=16 bf16, forward slab groups in sequence (1 GiB default
+    workspace): sampled rows of two heads and sampled keys of one head."""
     x = make_inputs(1, 16, 16384, 128, seed=4, dtype="bf16")
-    info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, True,
-                             rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, True))
-    assert info["groups"] > 1  # the slab is processed group by group
+    info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, False,
+                             rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, False))
+    assert info["groups"] > 1  # the forward's slab is processed group by group
     got = run(x, 16, False)
     rows = sample(16384, 4, edges=(0, 1, 1023, 1024))
     check_sampled(orc, x, got, False, [(0, 0), (0, 13)], rows, keys=sample(16384, 40, n=24))
@@ -232,14 +232,19 @@ def test_edge_shapes_f32(orc, shape, causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_row_range_groups(orc, dtype, causal):
     """A small workspace budget forces groups of 128-row ranges of one head (the last one
-    ragged), with dK/dV accumulated across groups."""
+    ragged): the forward's slab, and on the fp32 path the backward's, with dK/dV accumulated
+    across groups. The bf16 backward keeps no slab and runs as one group."""
     d = 64
     B, H, L, N = 1, 2, 700, 7
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     budget = 300 * 1024
-    info = rsa.plan_describe(B, H, L, d, N, causal, tdt, True,
-                             rsa.workspace_size(B, H, L, d, N, causal, tdt, True, budget))
-    assert info["rows_per_group"] < L and info["groups"] > B * H
+    for bwd in (False, True):
+        info = rsa.plan_describe(B, H, L, d, N, causal, tdt, bwd,
+                                 rsa.workspace_size(B, H, L, d, N, causal, tdt, bwd, budget))
+        if bwd and dtype == "bf16":
+            assert info["groups"] == 1
+        else:
+            assert info["rows_per_group"] < L and info["groups"] > B * H
     x = make_inputs(B, H, L, d, seed=300 + int(causal), dtype=dtype)
     got = run(x, N, causal, ws_budget=budget)
     check_full(orc, x, got, causal)
