@@ -82,13 +82,12 @@ def kernel_model(w):
         "qk_slab": (2 * p * d, 4 * p + 2 * t),                 # S fp32 write; Q, K read
         "slab_softmax": (0, 4 * p + 2 * p + row),               # S read, P bf16 write, lse
         "pv_ring_rows": (2 * p * d, 2 * p + 2 * t),             # P read, V read, O write
-        "rowdot": (0, 2 * t + row),
+        # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO O K V read,
+        # dQ write, lse read, the rows' lse*log2(e) and D written
+        "bwd_rows": (2 * p * d, 6 * t + 3 * row),
         # key-major backward: dP^T, dV, dK (+ the recomputed S^T, not counted); Q K V dO read,
-        # dK dV write, the rows' lse and D read
+        # dK dV write, the rows' lse*log2(e) and D read
         "bwd_keys": (6 * p * d, 6 * t + 2 * row),
-        # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO K V read, dQ
-        # write, lse and D read
-        "bwd_rows": (2 * p * d, 5 * t + 2 * row),
     }
 
 

@@ -107,6 +107,15 @@ RSA_API rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, c
 RSA_API const char *rsa_status_string(rsa_status_t status);
 
 /*
+ * What the most recent RSA_ERR_CUDA returned on the calling thread came from: the CUDA or
+ * driver call that failed, its error name and code, and for a tensor-map encoding the shape
+ * it was given. Thread-local storage owned by the library, valid until the thread's next
+ * failing call; an empty string if there was none. Not part of the paper's method: a
+ * diagnostic of this library.
+ */
+RSA_API const char *rsa_last_error(void);
+
+/*
  * Status reported by kernels since the last call of this function on the current device:
  * RSA_OK, or RSA_ERR_TIMEOUT if a bounded wait inside a kernel gave up (that kernel then
  * returned early and its outputs are invalid). Synchronises `stream` and clears the status.

@@ -3,8 +3,9 @@
 // "Sequence Parallelism: Making 4D Parallelism Possible" (review page, "Proposed method")
 // runs the backward pass on the same ring as the forward. Seen from key chunk m, the ring
 // brings every query chunk n = (m - s) mod N in turn; this kernel takes that view for a tile
-// of 128 keys (K_m, V_m resident in shared memory) and visits the group's query rows in
-// 64-row blocks, starting at the block of its own chunk and wrapping around:
+// of 128 keys (K_m, V_m resident on the chip: in TMEM for d = 64, in shared memory for
+// d = 128) and visits the query rows in 64-row blocks, starting at the block of its own chunk
+// and wrapping around:
 //
 //   S^T  = K_m Q_n^T,   dP^T = V_m dO_n^T                   (tcgen05, TMEM accumulators)
 //   P^T  = exp(scale S^T - lse_n),  dS^T = P^T (dP^T - D_n)   (epilogue warps, fp32 -> bf16)
@@ -51,6 +52,12 @@ struct BkCfg {
     // TMEM columns: S^T[b] at 128 b, dP^T[b] at 128 b + 64, dV at 256, dK at 256 + D.
     // P^T / dS^T of step t (bf16 pairs) overwrite S^T[b] / dP^T[b]: queries 32h..32h+31 of
     // step t occupy columns 32h .. 32h + 15 of the buffer.
+    // For d = 64 the unit's K and V tiles are also copied into TMEM (bf16 pairs, 32 columns
+    // each, at T_K and T_V) and the S^T / dP^T MMAs take their A operand from there, which
+    // halves their shared-memory traffic; for d = 128 the columns are all taken.
+    static constexpr bool KV_TMEM = D == 64;
+    static constexpr uint32_t T_K = 256 + 2 * D, T_V = T_K + D / 2;
+    static_assert(!KV_TMEM || T_V + D / 2 <= TMEM_COLS, "TMEM columns");
 };
 
 struct BkCtl {
@@ -280,6 +287,16 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
                 const uint32_t vs = ks + C::KV_BYTES;
                 const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, vs);
+                if (C::KV_TMEM) {
+                    // K, V -> TMEM (after the previous unit's S^T/dP^T MMAs, in issue order);
+                    // the shared-memory slot is free once the copies are done
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        tc_cp_128x256b(tmem + C::T_K + 8 * k, d_k + 2 * k);
+                        tc_cp_128x256b(tmem + C::T_V + 8 * k, d_v + 2 * k);
+                    }
+                    tc_commit(&ctl->kvempty[kv.stage]);
+                }
                 for (int s = 0; s < tl.cnt; ++s) {
                     const uint32_t b = gstep & 1u;
                     if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
@@ -292,17 +309,25 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     const uint32_t st = smem_addr(smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES);
                     const uint32_t t_s = tmem + 128 * b, t_p = t_s + 64;
                     const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
+                    if (C::KV_TMEM) {
 #pragma unroll
-                    for (int kb = 0; kb < D / 64; ++kb)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t en = (kb | k) != 0 ? 1u : 0u;
-                            const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
-                            tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
-                            tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
+                        for (int k = 0; k < D / 16; ++k) {
+                            tc_mma_bf16_ts(t_s, tmem + C::T_K + 8 * k, d_q + 2 * k, id_s, k ? 1u : 0u);
+                            tc_mma_bf16_ts(t_p, tmem + C::T_V + 8 * k, d_do + 2 * k, id_s, k ? 1u : 0u);
                         }
+                    } else {
+#pragma unroll
+                        for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t en = (kb | k) != 0 ? 1u : 0u;
+                                const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
+                                tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
+                                tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
+                            }
+                    }
                     tc_commit(&ctl->sfull[b]);
-                    if (s == tl.cnt - 1) tc_commit(&ctl->kvempty[kv.stage]);
+                    if (!C::KV_TMEM && s == tl.cnt - 1) tc_commit(&ctl->kvempty[kv.stage]);
                     if (pend && !grad()) {
                         ok = false;
                         break;
@@ -446,7 +471,9 @@ __global__ void __launch_bounds__(kBkThreads, 1)
 //
 // S and dP are recomputed instead of read back from the key-major kernel: the extra MMA work
 // costs less than a dS slab round trip through HBM. Each thread of the epilogue owns one query
-// row, so its statistics lse_i and D_i are two registers.
+// row, so its statistics lse_i and D_i are two registers. D_i = dO_i . O_i is formed here, from
+// the O tile loaded with Q and dO, and written out (with lse_i log2(e)) for the key-major
+// kernel, which runs next.
 //
 // Roles (320 threads) as in the key-major kernel: warp 0 lane 0 issues TMA loads, warp 1
 // owns TMEM and lane 0 issues tcgen05.mma, warps 2..9 are the epilogue (TMEM lanes
@@ -466,18 +493,19 @@ template <int D>
 struct BrCfg {
     static constexpr int KN = D == 64 ? 128 : 64;        // keys per step
     static constexpr int QT_BYTES = 128 * D * 2;         // [128 queries][D] tile
-    static constexpr int STAT_OFF = 2 * QT_BYTES;        // lse*log2(e) [128], then D [128]
-    static constexpr int SLOT_BYTES = 2 * QT_BYTES + 1024;
-    static constexpr int Q_SLOTS = 2;
+    static constexpr int SLOT_BYTES = 3 * QT_BYTES;      // Q, dO, O tiles of the unit
+    // one slot: it is free again once Q and dO are in TMEM and D is formed, early in a unit
+    static constexpr int Q_SLOTS = 1;
     static constexpr int KB_BYTES = KN * D * 2;          // [KN keys][D] block
     static constexpr int KCHUNK = KN * 128;              // one 64-column box of a block
     static constexpr int STAGE_BYTES = 2 * KB_BYTES;     // K block, V block
-    static constexpr int STAGES = D == 64 ? 3 : 2;
+    static constexpr int STAGES = D == 64 ? 4 : 3;
     static constexpr int OUT_BUFS = D == 64 ? 2 : 1;     // 2 KB staging buffers per warp
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_STAGE = OFF_Q + Q_SLOTS * SLOT_BYTES;
     static constexpr int OFF_OUT = OFF_STAGE + STAGES * STAGE_BYTES;
-    static constexpr int OFF_CTL = OFF_OUT + kEpiWarps * OUT_BUFS * 2048;
+    static constexpr int OFF_PART = OFF_OUT + kEpiWarps * OUT_BUFS * 2048;  // [2][2][128] fp32
+    static constexpr int OFF_CTL = OFF_PART + 2048;
     static constexpr uint32_t TMEM_COLS = 512;
     // TMEM columns: S[b] at KN b, dP at 2 KN, dQ at 3 KN, then the unit's Q and dO as bf16
     // pairs (the A operands of the S and dP MMAs, D / 2 columns each). dS of a step (bf16
@@ -488,11 +516,12 @@ struct BrCfg {
 
 struct BrCtl {
     uint64_t full[8], empty[8];    // K/V block stages
-    uint64_t qfull[2], qempty[2];  // resident Q/dO/statistics slots
+    uint64_t qfull[2], qempty[2];  // resident Q/dO/O slots
     uint64_t sfull[2];             // S[b] and dP computed
     uint64_t dpfree;               // dP loaded by every epilogue warp
     uint64_t pready[2];            // dS of buffer b written to TMEM
     uint64_t accfull, accempty;    // dQ accumulator
+    uint64_t dpair[4];             // both warps of rows 32q .. 32q + 31 posted their D partials
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -547,9 +576,10 @@ __device__ __forceinline__ void br_compute(const uint32_t (&rs)[32], const uint3
 template <int D>
 __global__ void __launch_bounds__(kBrThreads, 1)
     bwd_rows_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mdO,
-                    const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
-                    const __grid_constant__ CUtensorMap mStat,
-                    const __grid_constant__ CUtensorMap mdQ, const SlabArgs a) {
+                    const __grid_constant__ CUtensorMap mO, const __grid_constant__ CUtensorMap mK,
+                    const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mdQ,
+                    const float *__restrict__ lse, float *__restrict__ lse2_out,
+                    float *__restrict__ d_out, const SlabArgs a) {
     using C = BrCfg<D>;
     constexpr int KN = C::KN;
     extern __shared__ uint8_t smem_raw[];
@@ -565,7 +595,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         for (int s = 0; s < C::Q_SLOTS; ++s) {
             mbar_init(&ctl->qfull[s], 1);
             // released by the copies of Q and dO into TMEM and by every epilogue warp once
-            // it holds the rows' statistics in registers
+            // it has formed its rows' D from the dO and O tiles
             mbar_init(&ctl->qempty[s], 1 + kEpiWarps);
         }
         for (int b = 0; b < 2; ++b) {
@@ -573,6 +603,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             mbar_init(&ctl->pready[b], kEpiWarps);
         }
         mbar_init(&ctl->dpfree, kEpiWarps);
+        for (int w = 0; w < 4; ++w) mbar_init(&ctl->dpair[w], 2);
         mbar_init(&ctl->accfull, 1);
         mbar_init(&ctl->accempty, kEpiWarps);
         mbar_init(&ctl->drain, 1);
@@ -580,9 +611,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         fence_mbar_init();
         prefetch_tmap(&mQ);
         prefetch_tmap(&mdO);
+        prefetch_tmap(&mO);
         prefetch_tmap(&mK);
         prefetch_tmap(&mV);
-        prefetch_tmap(&mStat);
         prefetch_tmap(&mdQ);
     }
     if (warp == 1) {
@@ -613,14 +644,13 @@ __global__ void __launch_bounds__(kBrThreads, 1)
                 {
                     uint8_t *slot = smem + C::OFF_Q + qs.stage * C::SLOT_BYTES;
                     uint64_t *bar = &ctl->qfull[qs.stage];
-                    mbar_arrive_expect_tx(bar, 2 * C::QT_BYTES + 1024);
+                    mbar_arrive_expect_tx(bar, C::SLOT_BYTES);
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb) {
                         tma_load_3d(slot + kb * 16384, &mQ, bar, kb * 64, tl.i0, bh);
                         tma_load_3d(slot + C::QT_BYTES + kb * 16384, &mdO, bar, kb * 64, tl.i0, bh);
+                        tma_load_3d(slot + 2 * C::QT_BYTES + kb * 16384, &mO, bar, kb * 64, tl.i0, bh);
                     }
-                    tma_load_3d(slot + C::STAT_OFF, &mStat, bar, tl.i0, bh, 0);        // lse * log2(e)
-                    tma_load_3d(slot + C::STAT_OFF + 512, &mStat, bar, tl.i0, bh, 1);  // D
                     qissued[qs.stage] = true;
                     qpar[qs.stage] = qs.phase;
                     pipe_next(qs, C::Q_SLOTS);
@@ -755,23 +785,53 @@ __global__ void __launch_bounds__(kBrThreads, 1)
         const float sl2 = a.scale * kLog2e;
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
-        uint32_t gstep = 0, acc_ph = 0;
+        float *part = reinterpret_cast<float *>(smem + C::OFF_PART);
+        uint32_t gstep = 0, acc_ph = 0, unit = 0;
         int obuf = 0;
         Pipe qs{0, 0};
         bool ok = true;
-        for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
+        for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x, ++unit) {
             BrTile tl;
             br_decode(a, t, KN, tl);
             const int bh = a.bh0 + tl.h;
+            const int rt = 32 * q + lane;    // this thread's row of the tile
             const int iw = tl.i0 + 32 * q;  // this warp's first query row
             const int i = iw + lane;         // this thread's query row
+            const float lse_i = i < a.L ? lse[static_cast<size_t>(bh) * a.L + i] : 0.f;
             if (!warp_wait(&ctl->qfull[qs.stage], qs.phase, &ctl->abort)) break;
-            const float *stat = reinterpret_cast<const float *>(
-                smem + C::OFF_Q + qs.stage * C::SLOT_BYTES + C::STAT_OFF);
-            const float lse2 = stat[32 * q + lane], Di = stat[128 + 32 * q + lane];
+            // D_i = dO_i . O_i: this warp's half of the columns, then the other half's partial
+            // through shared memory (rows past L are zero-filled, so their D is 0)
+            const uint8_t *slot = smem + C::OFF_Q + qs.stage * C::SLOT_BYTES;
+            float dpart = 0.f;
+#pragma unroll
+            for (int g = hf * (D / 16); g < (hf + 1) * (D / 16); ++g) {
+                const uint32_t off = (g >> 3) * 16384 + sw128_offset(rt, g & 7);
+                const uint4 x = *reinterpret_cast<const uint4 *>(slot + C::QT_BYTES + off);
+                const uint4 y = *reinterpret_cast<const uint4 *>(slot + 2 * C::QT_BYTES + off);
+                const __nv_bfloat162 *xb = reinterpret_cast<const __nv_bfloat162 *>(&x);
+                const __nv_bfloat162 *yb = reinterpret_cast<const __nv_bfloat162 *>(&y);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 u = __bfloat1622float2(xb[e]), w = __bfloat1622float2(yb[e]);
+                    dpart = fmaf(u.x, w.x, dpart);
+                    dpart = fmaf(u.y, w.y, dpart);
+                }
+            }
+            float *pb = part + (unit & 1u) * 256;
+            pb[hf * 128 + rt] = dpart;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->dpair[q]);
+            if (!warp_wait(&ctl->dpair[q], unit & 1u, &ctl->abort)) break;
+            const float Di = dpart + pb[(hf ^ 1) * 128 + rt];
+            const float lse2 = lse_i * kLog2e;
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->qempty[qs.stage]);
             pipe_next(qs, C::Q_SLOTS);
+            // the rows' statistics for the key-major kernel, padded with zeros to Lp
+            if (hf == 0 && i < a.Lp) {
+                lse2_out[static_cast<size_t>(bh) * a.Lp + i] = lse2;
+                d_out[static_cast<size_t>(bh) * a.Lp + i] = Di;
+            }
             for (int s = 0; s < tl.cnt; ++s) {
                 const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
                 const int jw = ring_block(tl.first, s, tl.cnt) * KN + hf * (KN / 2);  // first key
@@ -884,16 +944,16 @@ cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const 
                       mV, mQ, mdO, mStat, mdK, mdV, a);
 }
 
-cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mK,
-                            const CUtensorMap &mV, const CUtensorMap &mStat,
-                            const CUtensorMap &mdQ, const SlabArgs &a, int num_sms,
-                            cudaStream_t st) {
+cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mO,
+                            const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mdQ,
+                            const float *lse, float *lse2_out, float *d_out, const SlabArgs &a,
+                            int num_sms, cudaStream_t st) {
     const int grid = tc::grid_for(a.ntiles, num_sms);
     if (a.d == 64)
         return launch_pdl(bwd_rows_kernel<64>, dim3(grid), dim3(kBrThreads), br_smem<64>(), st,
-                          mQ, mdO, mK, mV, mStat, mdQ, a);
+                          mQ, mdO, mO, mK, mV, mdQ, lse, lse2_out, d_out, a);
     return launch_pdl(bwd_rows_kernel<128>, dim3(grid), dim3(kBrThreads), br_smem<128>(), st, mQ,
-                      mdO, mK, mV, mStat, mdQ, a);
+                      mdO, mO, mK, mV, mdQ, lse, lse2_out, d_out, a);
 }
 
 }  // namespace rsa

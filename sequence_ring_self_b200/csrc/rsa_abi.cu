@@ -11,6 +11,7 @@
 
 #include <math.h>
 #include <mutex>
+#include <stdio.h>
 #include <string.h>
 #include <vector>
 
@@ -31,6 +32,18 @@ constexpr size_t kDefaultBudget = size_t(1) << 30;
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// What the last RSA_ERR_CUDA of the calling thread came from (see rsa_last_error).
+thread_local char g_err[320];
+
+rsa_status_t cuda_fail(const char *what, int code, const char *name) {
+    snprintf(g_err, sizeof(g_err), "%s failed: %s (%d)", what, name ? name : "?", code);
+    return RSA_ERR_CUDA;
+}
+
+rsa_status_t cuda_fail(const char *what, cudaError_t e) {
+    return cuda_fail(what, static_cast<int>(e), cudaGetErrorName(e));
+}
 
 struct Plan {
     int B, H, L, d, N, causal, bwd;
@@ -172,21 +185,28 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 rsa_status_t device_state(DeviceState **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return RSA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     if (dev < 0 || dev >= kMaxDevices) return RSA_ERR_UNSUPPORTED;
+    // make the device's primary context current on this thread: the tensor maps are encoded
+    // through the driver API, which needs one, possibly before any launch of this thread
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail("cudaSetDevice", e);
     std::lock_guard<std::mutex> lock(g_mutex);
     DeviceState &s = g_dev[dev];
     if (!s.ready) {
         int major = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-            return RSA_ERR_CUDA;
+        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
         if (major != 10) return RSA_ERR_UNSUPPORTED;
-        if (cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return RSA_ERR_CUDA;
-        if (rsa::tc_kernels_configure() != cudaSuccess || rsa::bwd_kernels_configure() != cudaSuccess)
-            return RSA_ERR_CUDA;
+        e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+        if ((e = rsa::tc_kernels_configure()) != cudaSuccess ||
+            (e = rsa::bwd_kernels_configure()) != cudaSuccess)
+            return cuda_fail("cudaFuncSetAttribute", e);
         void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, rsa::g_status_word) != cudaSuccess) return RSA_ERR_CUDA;
+        e = cudaGetSymbolAddress(&ptr, rsa::g_status_word);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress", e);
         s.status = static_cast<int *>(ptr);
         if (!g_encode) {
             void *fn = nullptr;
@@ -194,7 +214,7 @@ rsa_status_t device_state(DeviceState **out) {
             if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
                     cudaSuccess ||
                 q != cudaDriverEntryPointSuccess || !fn)
-                return RSA_ERR_CUDA;
+                return cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", 0, nullptr);
             g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         }
         s.ready = true;
@@ -249,12 +269,16 @@ rsa_status_t timed(int kind, cudaStream_t s, F &&launch) {
         std::lock_guard<std::mutex> lock(g_prof_mutex);
         a = pool_event();
         b = pool_event();
-        if (!a || !b || cudaEventRecord(a, s) != cudaSuccess) return RSA_ERR_CUDA;
+        if (!a || !b) return cuda_fail("cudaEventCreate", 0, nullptr);
+        const cudaError_t e = cudaEventRecord(a, s);
+        if (e != cudaSuccess) return cuda_fail("cudaEventRecord", e);
     }
-    if (launch() != cudaSuccess) return RSA_ERR_CUDA;
+    const cudaError_t e = launch();
+    if (e != cudaSuccess) return cuda_fail(kKindNames[kind], e);
     if (a) {
         std::lock_guard<std::mutex> lock(g_prof_mutex);
-        if (cudaEventRecord(b, s) != cudaSuccess) return RSA_ERR_CUDA;
+        const cudaError_t e2 = cudaEventRecord(b, s);
+        if (e2 != cudaSuccess) return cuda_fail("cudaEventRecord", e2);
         g_prof.push_back({kind, a, b});
     }
     return RSA_OK;
@@ -277,7 +301,15 @@ bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t 
     CUresult r = g_encode(m, type, 3, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_err, sizeof(g_err),
+                 "cuTensorMapEncodeTiled failed (%d): base %p dims %llu x %llu x %llu box %u x %u",
+                 static_cast<int>(r), base, static_cast<unsigned long long>(d0),
+                 static_cast<unsigned long long>(d1), static_cast<unsigned long long>(d2), box0,
+                 box1);
+        return false;
+    }
+    return true;
 }
 
 // Input tensor [BH][L][d] bf16, box of 64 columns x `rows` rows.
@@ -304,9 +336,10 @@ SlabArgs slab_args(const Plan &p, const Group &G, int *status) {
     return a;
 }
 
-#define RSA_TRY(expr)                            \
-    do {                                         \
-        if ((expr) != cudaSuccess) return RSA_ERR_CUDA; \
+#define RSA_TRY(expr)                                          \
+    do {                                                       \
+        const cudaError_t e_ = (expr);                         \
+        if (e_ != cudaSuccess) return cuda_fail(#expr, e_);    \
     } while (0)
 
 rsa_status_t check_common(const Plan &p, void *ws, size_t ws_bytes) {
@@ -353,6 +386,8 @@ rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rs
     out[4] = static_cast<long long>(p.total);
     return p.total > ws_bytes ? RSA_ERR_WORKSPACE : RSA_OK;
 }
+
+const char *rsa_last_error(void) { return g_err; }
 
 rsa_status_t rsa_profile_enable(int on) {
     std::lock_guard<std::mutex> lock(g_prof_mutex);
@@ -480,9 +515,10 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
     float *Dvec = lse2 + size_t(p.BH) * p.Lp;
     const float scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
 
-    // D_i = dO_i . O_i and lse_i * log2(e), in rows padded to Lp
-    RSA_LAUNCH(K_ROWDOT, rsa::launch_rowdot(dO, O, lse, Dvec, dt == RSA_BF16 ? lse2 : nullptr, p.BH,
-                                            L, p.Lp, d, dt == RSA_BF16, s));
+    if (dt == RSA_F32) {
+        // D_i = dO_i . O_i, in rows padded to Lp
+        RSA_LAUNCH(K_ROWDOT, rsa::launch_rowdot(dO, O, lse, Dvec, nullptr, p.BH, L, p.Lp, d, 0, s));
+    }
 
     if (dt == RSA_F32) {
         for (long long g = 0; g < p.ngroups; ++g) {
@@ -503,34 +539,33 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
         return RSA_OK;
     }
 
-    // Two kernels over the whole problem (one group): the key-major ring gives dK and dV,
-    // the query-major ring gives dQ; both recompute S and dP tile by tile from Q, K, V, dO
-    // and the row statistics, so nothing but the statistics goes through HBM.
-    CUtensorMap mK128, mV128, mQ64, mdO64, mStat64, mQ128, mdO128, mK64, mV64, mStat128;
+    // Two kernels over the whole problem (one group): the query-major ring gives dQ (and the
+    // rows' D and lse * log2(e)), then the key-major ring gives dK and dV; both recompute S and
+    // dP tile by tile from Q, K, V, dO and the row statistics, so nothing but the statistics
+    // goes through HBM.
+    CUtensorMap mK128, mV128, mQ64, mdO64, mStat64, mQ128, mdO128, mO128, mK64, mV64;
     CUtensorMap mdQ, mdK, mdV;
     const uint64_t stat_pitch = uint64_t(p.Lp) * 4;
     if (!map_input(&mK128, K, p, 128) || !map_input(&mV128, V, p, 128) ||
         !map_input(&mQ64, Q, p, 64) || !map_input(&mdO64, dO, p, 64) ||
         !map_input(&mQ128, Q, p, 128) || !map_input(&mdO128, dO, p, 128) ||
-        !map_input(&mK64, K, p, 64) || !map_input(&mV64, V, p, 64) ||
+        !map_input(&mO128, O, p, 128) || !map_input(&mK64, K, p, 64) ||
+        !map_input(&mV64, V, p, 64) ||
         !map3d(&mStat64, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2, p.Lp, p.BH, 2, stat_pitch,
                stat_pitch * p.BH, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !map3d(&mStat128, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2, p.Lp, p.BH, 2, stat_pitch,
-               stat_pitch * p.BH, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !map_output(&mdQ, dQ, p) || !map_output(&mdK, dK, p) || !map_output(&mdV, dV, p))
         return RSA_ERR_CUDA;
     const Group G = group_of(p, 0);
     SlabArgs a = slab_args(p, G, dev->status);
-    // key-major ring: P^T, dP^T -> dS^T in TMEM; dV_m, dK_m over all query blocks
     a.mode = 0;
     a.ntiles = G.nh * ((L + 127) / 128);
-    RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat64, mdK, mdV, a,
-                                                dev->sms, s));
     // query-major ring: S, dP -> dS in TMEM; dQ_n = scale * sum_m dS_nm K_m
-    a.ntiles = G.nh * ((L + 127) / 128);
     // (blocks of 128 keys for d = 64, of 64 keys for d = 128)
     const CUtensorMap &mKr = d == 64 ? mK128 : mK64, &mVr = d == 64 ? mV128 : mV64;
-    RSA_LAUNCH(K_BWD_ROWS, rsa::launch_bwd_rows(mQ128, mdO128, mKr, mVr, mStat128, mdQ, a,
+    RSA_LAUNCH(K_BWD_ROWS, rsa::launch_bwd_rows(mQ128, mdO128, mO128, mKr, mVr, mdQ, lse, lse2,
+                                                Dvec, a, dev->sms, s));
+    // key-major ring: P^T, dP^T -> dS^T in TMEM; dV_m, dK_m over all query blocks
+    RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat64, mdK, mdV, a,
                                                 dev->sms, s));
     return RSA_OK;
 }

@@ -65,14 +65,16 @@ cudaError_t launch_bwd_keys(const CUtensorMap &mK, const CUtensorMap &mV, const 
                             const CUtensorMap &mdO, const CUtensorMap &mStat,
                             const CUtensorMap &mdK, const CUtensorMap &mdV, const SlabArgs &a,
                             int num_sms, cudaStream_t st);
-// Row-major backward: recompute S, dP -> dS in TMEM per 128-query tile and dQ = scale dS K.
-// mQ/mdO: 64 x 128 boxes; mK/mV: 64 x 128 boxes for d = 64, 64 x 64 for d = 128 (the key
-// block of a step); mStat: as above with 128 x 1 x 1 boxes;
-// mdQ: [BH][L][d] bf16, 32 x 32 boxes, 64-byte swizzle (store).
-cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mK,
-                            const CUtensorMap &mV, const CUtensorMap &mStat,
-                            const CUtensorMap &mdQ, const SlabArgs &a, int num_sms,
-                            cudaStream_t st);
+// Row-major backward: recompute S, dP -> dS in TMEM per 128-query tile and dQ = scale dS K;
+// forms D_i = dO_i . O_i and writes lse_i log2(e) and D_i to lse2_out / d_out ([BH][Lp] each,
+// zero past L) for launch_bwd_keys, which must run after it.
+// mQ/mdO/mO: 64 x 128 boxes; mK/mV: 64 x 128 boxes for d = 64, 64 x 64 for d = 128 (the key
+// block of a step); mdQ: [BH][L][d] bf16, 32 x 32 boxes, 64-byte swizzle (store);
+// lse: [BH][L] fp32 from the forward pass.
+cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const CUtensorMap &mO,
+                            const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mdQ,
+                            const float *lse, float *lse2_out, float *d_out, const SlabArgs &a,
+                            int num_sms, cudaStream_t st);
 cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
 cudaError_t bwd_kernels_configure();
 

@@ -27,7 +27,7 @@ RSA_F32, RSA_BF16 = 0, 1
 EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
             "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
-            "rsa_forward_noalloc")
+            "rsa_forward_noalloc", "rsa_last_error")
 
 _lib = None
 _lock = threading.Lock()
@@ -36,7 +36,12 @@ _lock = threading.Lock()
 class RSAError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {status_string(code)} ({code})")
+        msg = f"{what}: {status_string(code)} ({code})"
+        if code == RSA_ERR_CUDA:
+            detail = load_library().rsa_last_error().decode(errors="replace")
+            if detail:
+                msg += f" [{detail}]"
+        super().__init__(msg)
 
 
 def load_library(path: str | None = None):
@@ -60,6 +65,8 @@ def load_library(path: str | None = None):
         lib.rsa_backward.restype = i
         lib.rsa_status_string.argtypes = [i]
         lib.rsa_status_string.restype = ctypes.c_char_p
+        lib.rsa_last_error.argtypes = []
+        lib.rsa_last_error.restype = ctypes.c_char_p
         lib.rsa_last_device_status.argtypes = [vp]
         lib.rsa_last_device_status.restype = i
         lib.rsa_plan_describe.argtypes = [i, i, i, i, i, i, i, i, sz, ctypes.POINTER(ctypes.c_longlong)]

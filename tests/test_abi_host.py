@@ -67,6 +67,15 @@ def test_argument_errors_are_reported_before_any_launch(lib, call):
     assert call(lib, ws=0) == rsa.RSA_ERR_INVALID_ARG
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a usable GPU")
+def test_cuda_failures_are_described(lib):
+    # valid arguments: without a GPU the call fails at its first CUDA call, and says which
+    assert _bwd(lib) == rsa.RSA_ERR_CUDA
+    assert b"failed" in lib.rsa_last_error()
+    with pytest.raises(rsa.RSAError, match="failed"):
+        raise rsa.RSAError(rsa.RSA_ERR_CUDA, "rsa_backward")
+
+
 def test_forward_rejects_null_lse(lib):
     assert _fwd(lib, lse=0) == rsa.RSA_ERR_INVALID_ARG
 

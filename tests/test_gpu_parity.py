@@ -12,6 +12,8 @@ not depend on the chunk count beyond rounding).
 """
 import types
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -292,6 +294,41 @@ def test_autograd_wrapper_and_host_api(orc):
     torch.cuda.synchronize()
     for n in ("O", "lse", "dQ", "dK", "dV"):
         np.testing.assert_array_equal(res[n].to(torch.float64).numpy(), ref[n])
+
+
+def test_calls_from_a_fresh_thread():
+    """A thread that has made no CUDA call yet (as autograd's backward thread may be) can call
+    the library: it binds the device's context itself before encoding its tensor maps."""
+    import threading
+    x = make_inputs(1, 2, 256, 64, seed=9, dtype="bf16")
+    ref = run(x, 4, False)
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+    o, lse = torch.empty_like(q), torch.empty(1, 2, 256, dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    nf = rsa.workspace_size(1, 2, 256, 64, 4, False, torch.bfloat16, False)
+    nb = rsa.workspace_size(1, 2, 256, 64, 4, False, torch.bfloat16, True)
+    wf = torch.empty(nf, dtype=torch.uint8, device=dev)
+    wb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    lib = rsa.load_library()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = []
+
+    def body():
+        rc.append(lib.rsa_forward(p(q), p(k), p(v), p(o), p(lse), 1, 2, 256, 64, 4, 0, rsa.RSA_BF16,
+                                  p(wf), nf, None))
+        rc.append(lib.rsa_backward(p(q), p(k), p(v), p(o), p(do), p(lse), p(dq), p(dk), p(dv),
+                                   1, 2, 256, 64, 4, 0, rsa.RSA_BF16, p(wb), nb, None))
+        rc.append(lib.rsa_last_device_status(None))
+
+    th = threading.Thread(target=body)
+    th.start()
+    th.join()
+    assert rc == [rsa.RSA_OK] * 3, [rsa.status_string(c) for c in rc]
+    torch.cuda.synchronize()
+    for n, t in (("O", o), ("dQ", dq), ("dK", dk), ("dV", dv)):
+        np.testing.assert_array_equal(np64(t), ref[n])
 
 
 def test_library_errors_raise():
