@@ -80,8 +80,7 @@ def kernel_model(w):
     row = BH * L * 4    # one fp32 per row (lse, D)
     return {
         "qk_slab": (2 * p * d, 4 * p + 2 * t),                 # S fp32 write; Q, K read
-        "slab_softmax": (0, 4 * p + 2 * p + row),               # S read, P bf16 write, lse
-        "pv_ring_rows": (2 * p * d, 2 * p + 2 * t),             # P read, V read, O write
+        "pv_softmax": (2 * p * d, 4 * p + 2 * t + row),         # S read, V read, O, lse write
         # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO O K V read,
         # dQ write, lse read, the rows' lse*log2(e) and D written
         "bwd_rows": (2 * p * d, 6 * t + 3 * row),
@@ -484,7 +483,7 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["sweep"], default="bert")

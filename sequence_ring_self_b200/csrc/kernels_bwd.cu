@@ -107,28 +107,52 @@ __device__ __forceinline__ void epi_compute(const uint32_t (&rs)[32], const uint
                                             const float *stat, float sl2, int j, int ic, int L,
                                             int r_end, int causal, uint32_t (&wp)[16],
                                             uint32_t (&wd)[16]) {
+    if (!MASK) {
+        // packed pairs: the exponent, dP - D and the product each one instruction per pair
+        const float2 sl = make_float2(sl2, sl2);
 #pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 l4 = reinterpret_cast<const float4 *>(stat)[e4];
-        const float4 d4 = reinterpret_cast<const float4 *>(stat + 64)[e4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pv[4], sv[4];
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = reinterpret_cast<const float4 *>(stat)[e4];
+            const float4 d4 = reinterpret_cast<const float4 *>(stat + 64)[e4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u;
-            float p = fast_exp2(fmaf(__uint_as_float(rs[e]), sl2, -lv[u]));
-            if (MASK) {
-                const int i = ic + e;
-                p = (j >= L || i >= r_end || (causal && j > i)) ? 0.f : p;
+            for (int h = 0; h < 2; ++h) {
+                const int e = 4 * e4 + 2 * h;
+                const float2 nl = h ? make_float2(-l4.z, -l4.w) : make_float2(-l4.x, -l4.y);
+                const float2 dv = h ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+                const float2 x = ffma2(make_float2(__uint_as_float(rs[e]), __uint_as_float(rs[e + 1])),
+                                       sl, nl);
+                const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                const float2 g = fsub2(make_float2(__uint_as_float(rd[e]), __uint_as_float(rd[e + 1])),
+                                       dv);
+                const float2 ds = fmul2(p, g);
+                wp[e >> 1] = pack_bf16x2(p.x, p.y);
+                wd[e >> 1] = pack_bf16x2(ds.x, ds.y);
             }
-            pv[u] = p;
-            sv[u] = p * (__uint_as_float(rd[e]) - dv[u]);
         }
-        wp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
-        wp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
-        wd[2 * e4] = pack_bf16x2(sv[0], sv[1]);
-        wd[2 * e4 + 1] = pack_bf16x2(sv[2], sv[3]);
+    } else {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = reinterpret_cast<const float4 *>(stat)[e4];
+            const float4 d4 = reinterpret_cast<const float4 *>(stat + 64)[e4];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], sv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = 4 * e4 + u;
+                float p = fast_exp2(fmaf(__uint_as_float(rs[e]), sl2, -lv[u]));
+                if (MASK) {
+                    const int i = ic + e;
+                    p = (j >= L || i >= r_end || (causal && j > i)) ? 0.f : p;
+                }
+                pv[u] = p;
+                sv[u] = p * (__uint_as_float(rd[e]) - dv[u]);
+            }
+            wp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+            wp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+            wd[2 * e4] = pack_bf16x2(sv[0], sv[1]);
+            wd[2 * e4 + 1] = pack_bf16x2(sv[2], sv[3]);
+        }
     }
 }
 
@@ -248,7 +272,102 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && C::KV_TMEM) {
+            // d = 64: S^T/dP^T run two steps ahead of dV/dK. Every barrier poll of this thread
+            // waits for the MMAs it has in flight, so the loop polls once per step: pready(g),
+            // which the epilogue posts only once the Q/dO stage of step g + 2 has landed too.
+            constexpr uint64_t KM = sdesc_const(16, 1024);
+            constexpr uint64_t MN = sdesc_const(8192, 1024);
+            const uint32_t id_s = idesc_bf16_f32(128, C::QB, 0, 0);
+            const uint32_t id_g = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + D;
+            struct Cursor {
+                int t, s;
+                BkTile tl;
+                Pipe p;
+            };
+            auto seek = [&](Cursor &c) -> bool {  // first unit at or after c.t with work
+                for (; c.t < a.ntiles; c.t += gridDim.x)
+                    if (bk_decode(a, c.t, c.tl)) {
+                        c.s = 0;
+                        return true;
+                    }
+                return false;
+            };
+            auto advance = [&](Cursor &c) -> bool {
+                pipe_next(c.p, C::STAGES);
+                if (++c.s < c.tl.cnt) return true;
+                c.t += gridDim.x;
+                return seek(c);
+            };
+            Cursor is{static_cast<int>(blockIdx.x), 0, {}, {0, 0}};
+            Cursor gr = is;
+            bool has_is = seek(is), has_gr = seek(gr);
+            Pipe kv{0, 0};
+            uint32_t gi = 0, gg = 0, acc_ph = 0;
+            auto issue_s = [&]() -> bool {  // S^T, dP^T of the step under `is`, buffer gi & 1
+                if (is.s == 0) {
+                    // K, V -> TMEM (after every earlier S^T/dP^T MMA, in issue order)
+                    if (!mbar_wait(&ctl->kvfull[kv.stage], kv.phase, &ctl->abort)) return false;
+                    tc_fence_after();
+                    const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
+                    const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, ks + C::KV_BYTES);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        tc_cp_128x256b(tmem + C::T_K + 8 * k, d_k + 2 * k);
+                        tc_cp_128x256b(tmem + C::T_V + 8 * k, d_v + 2 * k);
+                    }
+                    tc_commit(&ctl->kvempty[kv.stage]);
+                    pipe_next(kv, C::KV_SLOTS);
+                }
+                // the first two stages are not vouched for by a pready
+                if (gi < 2 && !mbar_wait(&ctl->full[is.p.stage], is.p.phase, &ctl->abort))
+                    return false;
+                tc_fence_after();
+                const uint32_t st = smem_addr(smem + C::OFF_STAGE + is.p.stage * C::STAGE_BYTES);
+                const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
+                const uint32_t t_s = tmem + 128 * (gi & 1u), t_p = t_s + 64;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    tc_mma_bf16_ts(t_s, tmem + C::T_K + 8 * k, d_q + 2 * k, id_s, k ? 1u : 0u);
+                    tc_mma_bf16_ts(t_p, tmem + C::T_V + 8 * k, d_do + 2 * k, id_s, k ? 1u : 0u);
+                }
+                tc_commit(&ctl->sfull[gi & 1u]);
+                ++gi;
+                has_is = advance(is);
+                return true;
+            };
+            bool ok = true;
+            if (has_is) ok = issue_s();
+            if (ok && has_is) ok = issue_s();
+            while (ok && has_gr) {
+                const uint32_t b = gg & 1u;
+                if (!mbar_wait(&ctl->pready[b], (gg >> 1) & 1u, &ctl->abort)) break;
+                const bool first = gr.s == 0, last = gr.s == gr.tl.cnt - 1;
+                if (first && !mbar_wait(&ctl->accempty, acc_ph ^ 1u, &ctl->abort)) break;
+                tc_fence_after();
+                const uint32_t st = smem_addr(smem + C::OFF_STAGE + gr.p.stage * C::STAGE_BYTES);
+                const uint64_t d_do = sdesc(MN, st + C::QT_BYTES), d_q = sdesc(MN, st);
+                const uint32_t t_p = tmem + 128 * b, t_ds = t_p + 64;
+#pragma unroll
+                for (int k = 0; k < C::QB / 16; ++k) {
+                    const uint32_t en = (first && k == 0) ? 0u : 1u;
+                    const uint32_t col = (k >> 1) * 32 + (k & 1) * 8;  // 16 queries per MMA
+                    tc_mma_bf16_ts(t_dv, t_p + col, d_do + 128 * k, id_g, en);
+                    tc_mma_bf16_ts(t_dk, t_ds + col, d_q + 128 * k, id_g, en);
+                }
+                tc_commit(&ctl->empty[gr.p.stage]);
+                if (last) {
+                    tc_commit(&ctl->accfull);
+                    acc_ph ^= 1u;
+                }
+                ++gg;
+                has_gr = advance(gr);
+                if (has_is) ok = issue_s();
+            }
+            tc_commit(&ctl->drain);
+            drain_wait(&ctl->drain, 0);
+        } else if (lane == 0) {
             constexpr uint64_t KM = sdesc_const(16, 1024);    // K-major, 128-byte swizzle
             constexpr uint64_t MN = sdesc_const(8192, 1024);  // MN-major, 64-wide blocks 8 KB apart
             const uint32_t id_s = idesc_bf16_f32(128, C::QB, 0, 0);  // S^T, dP^T
@@ -287,16 +406,6 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
                 const uint32_t vs = ks + C::KV_BYTES;
                 const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, vs);
-                if (C::KV_TMEM) {
-                    // K, V -> TMEM (after the previous unit's S^T/dP^T MMAs, in issue order);
-                    // the shared-memory slot is free once the copies are done
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        tc_cp_128x256b(tmem + C::T_K + 8 * k, d_k + 2 * k);
-                        tc_cp_128x256b(tmem + C::T_V + 8 * k, d_v + 2 * k);
-                    }
-                    tc_commit(&ctl->kvempty[kv.stage]);
-                }
                 for (int s = 0; s < tl.cnt; ++s) {
                     const uint32_t b = gstep & 1u;
                     if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
@@ -309,25 +418,17 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     const uint32_t st = smem_addr(smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES);
                     const uint32_t t_s = tmem + 128 * b, t_p = t_s + 64;
                     const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
-                    if (C::KV_TMEM) {
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            tc_mma_bf16_ts(t_s, tmem + C::T_K + 8 * k, d_q + 2 * k, id_s, k ? 1u : 0u);
-                            tc_mma_bf16_ts(t_p, tmem + C::T_V + 8 * k, d_do + 2 * k, id_s, k ? 1u : 0u);
+                    for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t en = (kb | k) != 0 ? 1u : 0u;
+                            const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
+                            tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
+                            tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
                         }
-                    } else {
-#pragma unroll
-                        for (int kb = 0; kb < D / 64; ++kb)
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint32_t en = (kb | k) != 0 ? 1u : 0u;
-                                const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
-                                tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
-                                tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
-                            }
-                    }
                     tc_commit(&ctl->sfull[b]);
-                    if (!C::KV_TMEM && s == tl.cnt - 1) tc_commit(&ctl->kvempty[kv.stage]);
+                    if (s == tl.cnt - 1) tc_commit(&ctl->kvempty[kv.stage]);
                     if (pend && !grad()) {
                         ok = false;
                         break;
@@ -360,6 +461,12 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         uint32_t gstep = 0, acc_ph = 0;
         Pipe ps{0, 0};  // the Q/dO stage of the current step (same order as the producer's)
         bool ok = true;
+        uint32_t total = 0;  // steps of this CTA (d = 64: pready(g) vouches for stage g + 2)
+        if (C::KV_TMEM)
+            for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+                BkTile tl;
+                if (bk_decode(a, t, tl)) total += tl.cnt;
+            }
         for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
             BkTile tl;
             if (!bk_decode(a, t, tl)) continue;
@@ -396,6 +503,15 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tmem_st16(t_s + 64, wd);
                 tmem_st_wait();
                 tc_fence_before();
+                if (C::KV_TMEM && gstep + 2 < total) {
+                    Pipe p2 = ps;
+                    pipe_next(p2, C::STAGES);
+                    pipe_next(p2, C::STAGES);
+                    if (!warp_wait(&ctl->full[p2.stage], p2.phase, &ctl->abort)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->pready[b]);
                 ++gstep;
@@ -557,19 +673,34 @@ template <bool MASK>
 __device__ __forceinline__ void br_compute(const uint32_t (&rs)[32], const uint32_t *rd, float sl2,
                                            float lse2, float Di, int j0, int i, int L, int causal,
                                            uint32_t (&wd)[16]) {
+    if (!MASK) {
+        // packed pairs: the exponent, dP - D and the product each one instruction per pair
+        const float2 sl = make_float2(sl2, sl2), nl = make_float2(-lse2, -lse2);
+        const float2 dd = make_float2(Di, Di);
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        float v[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            float p = fast_exp2(fmaf(__uint_as_float(rs[e + u]), sl2, -lse2));
-            if (MASK) {
-                const int j = j0 + e + u;
-                p = (j >= L || (causal && j > i)) ? 0.f : p;
-            }
-            v[u] = p * (__uint_as_float(rd[e + u]) - Di);
+        for (int e = 0; e < 32; e += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(rs[e]), __uint_as_float(rs[e + 1])),
+                                   sl, nl);
+            const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            const float2 g = fsub2(make_float2(__uint_as_float(rd[e]), __uint_as_float(rd[e + 1])), dd);
+            const float2 ds = fmul2(p, g);
+            wd[e >> 1] = pack_bf16x2(ds.x, ds.y);
         }
-        wd[e >> 1] = pack_bf16x2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            float v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                float p = fast_exp2(fmaf(__uint_as_float(rs[e + u]), sl2, -lse2));
+                if (MASK) {
+                    const int j = j0 + e + u;
+                    p = (j >= L || (causal && j > i)) ? 0.f : p;
+                }
+                v[u] = p * (__uint_as_float(rd[e + u]) - Di);
+            }
+            wd[e >> 1] = pack_bf16x2(v[0], v[1]);
+        }
     }
 }
 

@@ -1,12 +1,13 @@
 // kernels_simt.cu -- CUDA-core kernels of Ring Self-Attention.
 //
 //  * slab_softmax: the row softmax over the full key length that sits between the two ring
-//    passes ("Sequence Parallelism: Making 4D Parallelism Possible", review page, "Proposed
-//    method": attention is computed chunk by chunk with the keys passed around the ring).
-//    Each row of the fp32 score slab is read once with 16-byte loads and held in registers;
-//    max and sum use warp shuffles (plus shared memory across the row's warps). P is written
-//    in place: bf16 into the first half of the row's bytes, or fp32 over the scores.
-//  * rowdot: D_i = dO_i . O_i for the backward pass.
+//    passes of the fp32 path ("Sequence Parallelism: Making 4D Parallelism Possible", review
+//    page, "Proposed method": attention is computed chunk by chunk with the keys passed
+//    around the ring). Each row of the fp32 score slab is read once with 16-byte loads and
+//    held in registers; max and sum use warp shuffles (plus shared memory across the row's
+//    warps). P is written in place over the scores. (The bf16 path forms P inside its ring
+//    pass 2 kernel instead.)
+//  * rowdot: D_i = dO_i . O_i for the fp32 backward pass.
 //  * f32_*: the fp32 path, every step in fp32 FMA on the CUDA cores (no TF32), on the same
 //    slab layout and ring order as the tensor-core path.
 #include <cuda_bf16.h>
@@ -121,81 +122,6 @@ __global__ void __launch_bounds__(1024)
             reinterpret_cast<uint2 *>(row)[f] = w;
         } else {
             reinterpret_cast<float4 *>(row)[f] = make_float4(p0, p1, p2, p3);
-        }
-    }
-}
-
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ void combine2(float &m, float &l, float m2, float l2) {
-    const float nm = fmaxf(m, m2);
-    if (nm == -INFINITY) return;
-    l = l * ex2_approx(m - nm) + l2 * ex2_approx(m2 - nm);
-    m = nm;
-}
-
-// Streaming row softmax of the bf16 path. Scores are in base-2 units (s = log2(e) * scale *
-// q.k) and the slab GEMM left, per row and 128-column half tile, the partials (max, sum of
-// 2^(s - max)). One warp per row: combine the row's live partials, write lse = ln 2 *
-// (m + log2 l), then stream the row once, P = 2^(s - m) / l as bf16 into the first half of
-// the row's bytes. Each 512-column step loads before it stores (after __syncwarp), and later
-// steps only overwrite scores read by earlier ones, so the in-place write is safe.
-__global__ void __launch_bounds__(256)
-    slab_softmax_stream_kernel(float *__restrict__ slab, float *__restrict__ lse, const SlabArgs a) {
-    pdl_wait();
-    pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const long long nrows = static_cast<long long>(a.nh) * a.R;
-    const long long wstride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-    for (long long rid = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-         rid < nrows; rid += wstride) {
-        const int h = static_cast<int>(rid / a.R);
-        const int i = a.r0 + static_cast<int>(rid - static_cast<long long>(h) * a.R);
-        const int end = live_end(a, i);
-        const int nlive = a.causal ? 2 * ((min(a.L, (i / 128) * 128 + 128) + 255) / 256) : a.nStat;
-        const float2 *st = a.stats + rid * a.nStat;
-        float m = -INFINITY, l = 0.f;
-        for (int k = lane; k < nlive; k += 32) {
-            const float2 x = st[k];
-            combine2(m, l, x.x, x.y);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-            const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-            combine2(m, l, m2, l2);
-        }
-        if (lane == 0) lse[static_cast<size_t>(a.bh0 + h) * a.L + i] = (m + __log2f(l)) * 0.6931471805599453f;
-        const float inv = 1.f / l;
-        float *row = slab + rid * a.Lp;
-        for (int c0 = 0; c0 < end; c0 += 512) {
-            float4 x[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int c = c0 + 128 * u + 4 * lane;
-                x[u] = c < end ? reinterpret_cast<const float4 *>(row)[c >> 2]
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            uint2 w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float p0 = ex2_approx(x[u].x - m) * inv, p1 = ex2_approx(x[u].y - m) * inv;
-                const float p2 = ex2_approx(x[u].z - m) * inv, p3 = ex2_approx(x[u].w - m) * inv;
-                __nv_bfloat162 lo = __floats2bfloat162_rn(p0, p1);
-                __nv_bfloat162 hi = __floats2bfloat162_rn(p2, p3);
-                w[u].x = *reinterpret_cast<uint32_t *>(&lo);
-                w[u].y = *reinterpret_cast<uint32_t *>(&hi);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int c = c0 + 128 * u + 4 * lane;
-                if (c < end) reinterpret_cast<uint2 *>(row)[c >> 2] = w[u];
-            }
         }
     }
 }
@@ -545,14 +471,6 @@ cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int 
             e = launch_pdl(slab_softmax_kernel<32, false>, dim3((unsigned)grid), dim3(threads), 0, st, slab, lse, a, wpr);
     }
     return e;
-}
-
-cudaError_t launch_slab_softmax_stream(float *slab, float *lse, const SlabArgs &a, cudaStream_t st) {
-    const long long rows = static_cast<long long>(a.nh) * a.R;
-    long long grid = (rows + 7) / 8;
-    if (grid > 148LL * 32) grid = 148LL * 32;
-    return launch_pdl(slab_softmax_stream_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
-                      slab, lse, a);
 }
 
 cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,

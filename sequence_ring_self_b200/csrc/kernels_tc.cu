@@ -8,21 +8,19 @@
 // of tiles: each kernel below visits the key (or query) blocks of a tile starting at the
 // block of its own chunk and wrapping around, which is the ring rotation.
 //
-// Two kernels here (the backward's key-major kernel is in kernels_bwd.cu), persistent and
-// warp-specialised (192 threads = 6 warps):
+// The forward's two kernels (the backward's are in kernels_bwd.cu), persistent and
+// warp-specialised (320 threads = 10 warps):
 //   warp 0 lane 0 : TMA producer (global -> shared, 128-byte swizzle, mbarrier pipeline)
-//   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma into a double-buffered
-//                   TMEM accumulator and commits to mbarriers
-//   warps 2..5    : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (one tile row each)
+//   warp 1        : allocates TMEM; lane 0 issues tcgen05.mma and commits to mbarriers
+//   warps 2..9    : epilogue; warp w reads TMEM lanes 32*(w%4)..+31 (one tile row each)
 //
-//   qk_slab    (ring pass 1)      S = scale * Q K^T, masked, fp32 slab      A, B K-major
-//   ring_rows  (ring pass 2, dQ)  out = scale * A B over the slab's keys      B MN-major
+//   qk_slab     (ring pass 1)      S = scale * Q K^T, masked, fp32 slab + softmax partials
+//   pv_softmax  (softmax, pass 2)  P = softmax(S) formed on the chip, O = P V
 #include "tc_common.cuh"
 
 namespace rsa {
 namespace {
 
-constexpr int kThreads = 192;
 using namespace tc;
 
 // ======================================================================================
@@ -253,27 +251,61 @@ __global__ void __launch_bounds__(kQkThreads, 1)
 }
 
 // ======================================================================================
-// ring_rows: out[bh][i][:] = scale * sum_j P(i, j) * V[bh][j][:]   (bf16 out; ring pass 2)
-// P is the row-major bf16 slab P[h][i - r0][j], read K-major in 128 x 64 boxes. V ([L][D])
-// is the MN-major operand, read in 64-row boxes 64 columns wide. K-loop over 64-key blocks
-// in ring order starting at the tile's own chunk; causal tiles stop at their diagonal block.
+// pv_softmax: the row softmax and ring pass 2 in one kernel.
+//   P[i][j] = 2^(S[i][j] - m_i) / l_i,   O_i = sum over the ring of P[i][block m] V_m
+// where (m_i, l_i) combine the per-row partials that qk_slab left (max and sum of 2^(s - max)
+// per 128 key columns), and lse_i = ln 2 (m_i + log2 l_i) is written for the backward pass.
+// Work unit: (128-row tile, head), longest causal tiles first; the key blocks (64 keys) of a
+// unit are visited in ring order from the block of the tile's own chunk. Per step the
+// producer loads the fp32 score block (two 32-column boxes, 128 rows) and the V block; the
+// epilogue warps turn the scores into bf16 P in TMEM (keys 32g .. 32g + 31 of the block in
+// columns 16g .. 16g + 15 of the buffer) and the MMA thread accumulates O += P V with P as
+// the TMEM operand. P never goes back to HBM: the slab is read once, in fp32.
+// Roles (320 threads): warp 0 lane 0 TMA producer, warp 1 TMEM owner and MMA issuer,
+// warps 2..9 epilogue (TMEM lanes 32*(w%4)..+31 = rows; keys 32*((w-2)/4)..+31 of a block).
 // ======================================================================================
+constexpr int kPvThreads = 320;
+constexpr int kPvEpiWarps = 8;
+
 template <int D>
-struct RowsCfg {
-    static constexpr int A_BYTES = 128 * 64 * 2;
-    static constexpr int B_BYTES = 64 * D * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = D == 64 ? 6 : 5;
-    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + (int)sizeof(Ctl);
-    static constexpr uint32_t TMEM_COLS = D == 64 ? 128 : 256;
+struct PvCfg {
+    static constexpr int S_BYTES = 128 * 64 * 4;   // [128 rows][64 keys] fp32, two 16 KB boxes
+    static constexpr int V_BYTES = 64 * D * 2;     // [64 keys][D] bf16
+    static constexpr int STAGE_BYTES = S_BYTES + V_BYTES;
+    // d = 64: two CTAs per SM (2 stages each, 97 KB of shared memory and 256 TMEM columns
+    // apiece) so that twice the warps hide the latency of the streaming loads and of the
+    // barrier hand-offs; d = 128 does not fit twice and keeps one CTA with 4 stages
+    static constexpr int CTAS = D == 64 ? 2 : 1;
+    static constexpr int STAGES = D == 64 ? 2 : 4;
+    static constexpr int OUT_BUFS = 1;                // 2 KB staging buffer per warp
+    static constexpr int OFF_OUT = STAGES * STAGE_BYTES;
+    static constexpr int OFF_CTL = OFF_OUT + kPvEpiWarps * OUT_BUFS * 2048;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t T_O = 64;            // P[b] at 32 b (bf16 pairs), O at 64
+    static_assert(T_O + D <= TMEM_COLS, "TMEM columns");
 };
 
-struct RowsTile {
+struct PvCtl {
+    uint64_t full[8], empty[8];  // score / V stages
+    uint64_t pready[2];          // P of buffer b written to TMEM
+    uint64_t pfree[2];           // the MMAs that read P of buffer b are done
+    uint64_t accfull, accempty;  // O accumulator
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int D>
+constexpr int pv_smem() {
+    return 1024 + PvCfg<D>::OFF_CTL + static_cast<int>(sizeof(PvCtl));
+}
+
+struct PvTile {
     int h, i0, nkb, first;
 };
 
-// Tiles are (128-row tile, head), longest causal tiles first.
-__device__ __forceinline__ void rows_decode(const SlabArgs &a, int t, RowsTile &tl) {
+// Units are (128-row tile, head), longest causal tiles first.
+__device__ __forceinline__ void pv_decode(const SlabArgs &a, int t, PvTile &tl) {
     const int rt = a.nRT - 1 - t / a.nh;
     tl.h = t - (t / a.nh) * a.nh;
     tl.i0 = a.r0 + rt * 128;
@@ -283,21 +315,39 @@ __device__ __forceinline__ void rows_decode(const SlabArgs &a, int t, RowsTile &
     tl.first = min((n * a.c) / 64, tl.nkb - 1);
 }
 
+// 16-byte chunk g of row r in a [32 rows][64 bytes] staging tile, 64-byte swizzle.
+__device__ __forceinline__ uint32_t pv_sw64(uint32_t row, uint32_t g) {
+    return row * 64u + ((g ^ ((row >> 1) & 3u)) << 4);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    ring_rows_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                     __nv_bfloat16 *__restrict__ out, const SlabArgs a) {
-    using C = RowsCfg<D>;
+__global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
+    pv_softmax_kernel(const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mV,
+                      const __grid_constant__ CUtensorMap mO, float *__restrict__ lse,
+                      const SlabArgs a) {
+    using C = PvCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_1024(smem_raw);
-    uint8_t *stages = smem;
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem + C::STAGES * C::STAGE_BYTES);
+    PvCtl *ctl = reinterpret_cast<PvCtl *>(smem + C::OFF_CTL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        init_ctl(ctl, C::STAGES, 4);
-        prefetch_tmap(&mA);
-        prefetch_tmap(&mB);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->pready[b], kPvEpiWarps);
+            mbar_init(&ctl->pfree[b], 1);
+        }
+        mbar_init(&ctl->accfull, 1);
+        mbar_init(&ctl->accempty, kPvEpiWarps);
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&mS);
+        prefetch_tmap(&mV);
+        prefetch_tmap(&mO);
     }
     if (warp == 1) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
@@ -307,11 +357,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
-    // everything above (barriers, TMEM, descriptor prefetch) overlaps the previous kernel
     pdl_wait();
     pdl_trigger();
 
     if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             Pipe p{0, 0};
             bool issued[C::STAGES];
@@ -319,21 +369,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < C::STAGES; ++s) issued[s] = false, ipar[s] = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
-                RowsTile tl;
-                rows_decode(a, t, tl);
+                PvTile tl;
+                pv_decode(a, t, tl);
                 for (int s = 0; s < tl.nkb; ++s) {
-                    const int kb = ring_block(tl.first, s, tl.nkb);
+                    const int j0 = ring_block(tl.first, s, tl.nkb) * 64;
                     if (!mbar_wait(&ctl->empty[p.stage], p.phase ^ 1u, &ctl->abort)) {
                         ok = false;
                         break;
                     }
-                    uint8_t *sa = stages + p.stage * C::STAGE_BYTES;
+                    uint8_t *st = smem + p.stage * C::STAGE_BYTES;
                     uint64_t *bar = &ctl->full[p.stage];
                     mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                    tma_load_3d(sa, &mA, bar, kb * 64, tl.i0 - a.r0, tl.h);
+                    tma_load_3d(st, &mS, bar, j0, tl.i0 - a.r0, tl.h);
+                    tma_load_3d(st + 16384, &mS, bar, j0 + 32, tl.i0 - a.r0, tl.h);
 #pragma unroll
                     for (int dp = 0; dp < D / 64; ++dp)
-                        tma_load_3d(sa + C::A_BYTES + dp * 8192, &mB, bar, dp * 64, kb * 64,
+                        tma_load_3d(st + C::S_BYTES + dp * 8192, &mV, bar, dp * 64, j0,
                                     a.bh0 + tl.h);
                     issued[p.stage] = true;
                     ipar[p.stage] = p.phase;
@@ -345,79 +396,137 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            Pipe p{0, 0};
-            int acc = 0;
-            uint32_t aph = 0;
+            constexpr uint64_t MN = sdesc_const(8192, 1024);  // V: MN-major, 64-wide blocks
             const uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
-            constexpr uint64_t DA = sdesc_const(16, 1024);    // K-major P
-            constexpr uint64_t DB = sdesc_const(8192, 1024);  // MN-major V
-            constexpr uint32_t KSTEP_A = 2;  // 16 K-elements in 16-byte units
+            const uint32_t t_o = tmem + C::T_O;
+            Pipe p{0, 0};
+            uint32_t gstep = 0, acc_ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
-                RowsTile tl;
-                rows_decode(a, t, tl);
-                if (!mbar_wait(&ctl->tempty[acc], aph ^ 1u, &ctl->abort)) break;
-                tc_fence_after();
-                const uint32_t dcol = tmem + acc * D;
+                PvTile tl;
+                pv_decode(a, t, tl);
                 for (int s = 0; s < tl.nkb; ++s) {
-                    if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
+                    const uint32_t b = gstep & 1u;
+                    if (!mbar_wait(&ctl->pready[b], (gstep >> 1) & 1u, &ctl->abort) ||
+                        (s == 0 && !mbar_wait(&ctl->accempty, acc_ph ^ 1u, &ctl->abort))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(stages + p.stage * C::STAGE_BYTES);
-                    const uint64_t da = sdesc(DA, sa), db = sdesc(DB, sa + C::A_BYTES);
+                    const uint64_t dv = sdesc(MN, smem_addr(smem + p.stage * C::STAGE_BYTES + C::S_BYTES));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc_mma_bf16(dcol, da + KSTEP_A * k, db + 128 * k, idesc, (s | k) != 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)  // 16 keys per MMA, P columns 8k .. 8k + 7
+                        tc_mma_bf16_ts(t_o, tmem + 32 * b + 8 * k, dv + 128 * k, idesc,
+                                       (s | k) != 0 ? 1u : 0u);
                     tc_commit(&ctl->empty[p.stage]);
+                    tc_commit(&ctl->pfree[b]);
                     pipe_next(p, C::STAGES);
+                    ++gstep;
                 }
                 if (!ok) break;
-                tc_commit(&ctl->tfull[acc]);
-                acc ^= 1;
-                if (acc == 0) aph ^= 1u;
+                tc_commit(&ctl->accfull);
+                acc_ph ^= 1u;
             }
             tc_commit(&ctl->drain);
             drain_wait(&ctl->drain, 0);
         }
         __syncwarp();
     } else {
-        const int q = warp & 3;
-        int acc = 0;
-        uint32_t aph = 0;
-        for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-            RowsTile tl;
-            rows_decode(a, t, tl);
-            if (!warp_wait(&ctl->tfull[acc], aph, &ctl->abort)) break;
-            tc_fence_after();
-            const int i = tl.i0 + 32 * q + lane;
-            const bool row_ok = i < a.r0 + a.R;
-            __nv_bfloat16 *orow = out + (static_cast<size_t>(a.bh0 + tl.h) * a.L + i) * D;
-#pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * D + cc * 32, r);
-                tmem_ld_wait();
-                if (row_ok) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            w[u] = pack_bf16x2(__uint_as_float(r[8 * g + 2 * u]) * a.scale,
-                                               __uint_as_float(r[8 * g + 2 * u + 1]) * a.scale);
-                        st_global_v4(orow + cc * 32 + 8 * g, w[0], w[1], w[2], w[3]);
-                    }
+        // ------------------------------------------------------------------ epilogue
+        const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+        uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
+        uint32_t gstep = 0, acc_ph = 0;
+        int obuf = 0;
+        Pipe p{0, 0};
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
+            PvTile tl;
+            pv_decode(a, t, tl);
+            const int bh = a.bh0 + tl.h;
+            const int iw = tl.i0 + 32 * q;  // this warp's first row
+            const int i = iw + lane;         // this thread's row
+            // the row's softmax statistics from the slab GEMM's partials
+            float m = 0.f, inv = 0.f;
+            if (i < a.r0 + a.R) {
+                const int nlive =
+                    a.causal ? 2 * ((min(a.L, (i / 128) * 128 + 128) + 255) / 256) : a.nStat;
+                const float2 *st = a.stats + (static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat;
+                float l = 0.f;
+                m = -INFINITY;
+                for (int k = 0; k < nlive; ++k) {
+                    const float2 x = st[k];
+                    softmax_combine(m, l, x.x, x.y);
                 }
+                inv = 1.f / l;
+                if (hf == 0) lse[static_cast<size_t>(bh) * a.L + i] = (m + __log2f(l)) * 0.6931471805599453f;
             }
+            for (int s = 0; s < tl.nkb; ++s) {
+                const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
+                // scores of this step landed; P[b] is no longer read by the MMAs of step - 2
+                if (!warp_wait(&ctl->full[p.stage], p.phase, &ctl->abort) ||
+                    !warp_wait(&ctl->pfree[b], bph ^ 1u, &ctl->abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *sb = smem + p.stage * C::STAGE_BYTES + hf * 16384;
+                uint32_t w[16];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sb + sw128_offset(32 * q + lane, c));
+                    w[2 * c] = pack_bf16x2(fast_exp2(x.x - m) * inv, fast_exp2(x.y - m) * inv);
+                    w[2 * c + 1] = pack_bf16x2(fast_exp2(x.z - m) * inv, fast_exp2(x.w - m) * inv);
+                }
+                tc_fence_after();
+                tmem_st16(tmem + lane_base + 32 * b + 16 * hf, w);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->pready[b]);
+                pipe_next(p, C::STAGES);
+                ++gstep;
+            }
+            if (!ok) break;
+            // O of this tile, bf16, through the staging buffer
+            if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
+            acc_ph ^= 1u;
+            tc_fence_after();
+            uint32_t r[D / 64][32];
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc)
+                tmem_ld32(tmem + lane_base + C::T_O + hf * (D / 2) + 32 * cc, r[cc]);
+            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
-            acc ^= 1;
-            if (acc == 0) aph ^= 1u;
+            if (lane == 0) mbar_arrive(&ctl->accempty);
+            if (iw >= a.r0 + a.R) continue;  // the whole 32-row box lies past the group's rows
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                uint8_t *buf = obase + obuf * 2048;
+                obuf = obuf + 1 == C::OUT_BUFS ? 0 : obuf + 1;
+                if (lane == 0) bulk_wait_read<C::OUT_BUFS - 1>();
+                __syncwarp();
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = pack_bf16x2(__uint_as_float(r[cc][8 * g + 2 * u]),
+                                           __uint_as_float(r[cc][8 * g + 2 * u + 1]));
+                    *reinterpret_cast<uint4 *>(buf + pv_sw64(lane, g)) = make_uint4(v[0], v[1], v[2], v[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&mO, buf, hf * (D / 2) + 32 * cc, iw, bh);
+                    bulk_commit();
+                }
+            }
         }
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -442,8 +551,8 @@ cudaError_t tc_kernels_configure() {
     if (e != cudaSuccess) return e;
     RSA_SMEM(qk_slab_kernel<64>, QkCfg<64>::SMEM)
     RSA_SMEM(qk_slab_kernel<128>, QkCfg<128>::SMEM)
-    RSA_SMEM(ring_rows_kernel<64>, RowsCfg<64>::SMEM)
-    RSA_SMEM(ring_rows_kernel<128>, RowsCfg<128>::SMEM)
+    RSA_SMEM(pv_softmax_kernel<64>, pv_smem<64>())
+    RSA_SMEM(pv_softmax_kernel<128>, pv_smem<128>())
 #undef RSA_SMEM
     return cudaSuccess;
 }
@@ -459,15 +568,14 @@ cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const C
     return e;
 }
 
-cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
-                             const SlabArgs &a, int num_sms, cudaStream_t st) {
-    const int grid = tc::grid_for(a.ntiles, num_sms);
-    auto *o = static_cast<__nv_bfloat16 *>(out);
+cudaError_t launch_pv_softmax(const CUtensorMap &mS, const CUtensorMap &mV, const CUtensorMap &mO,
+                              float *lse, const SlabArgs &a, int num_sms, cudaStream_t st) {
+    const int grid = tc::grid_for(a.ntiles, num_sms * (a.d == 64 ? PvCfg<64>::CTAS : PvCfg<128>::CTAS));
     if (a.d == 64)
-        return launch_pdl(ring_rows_kernel<64>, dim3(grid), dim3(kThreads), RowsCfg<64>::SMEM,
-                          st, mA, mB, o, a);
-    return launch_pdl(ring_rows_kernel<128>, dim3(grid), dim3(kThreads), RowsCfg<128>::SMEM, st,
-                      mA, mB, o, a);
+        return launch_pdl(pv_softmax_kernel<64>, dim3(grid), dim3(kPvThreads), pv_smem<64>(), st,
+                          mS, mV, mO, lse, a);
+    return launch_pdl(pv_softmax_kernel<128>, dim3(grid), dim3(kPvThreads), pv_smem<128>(), st,
+                      mS, mV, mO, lse, a);
 }
 
 }  // namespace rsa

@@ -230,7 +230,7 @@ enum Kind {
     K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
-    "qk_slab", "slab_softmax", "pv_ring_rows", "rowdot", "bwd_keys", "bwd_rows",
+    "qk_slab", "slab_softmax", "pv_softmax", "rowdot", "bwd_keys", "bwd_rows",
     "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows"};
 
 struct ProfRec {
@@ -462,33 +462,30 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         return RSA_OK;
     }
 
-    CUtensorMap mQ, mK, mV;
-    if (!map_input(&mQ, Q, p, 128) || !map_input(&mK, K, p, 256) || !map_input(&mV, V, p, 64))
+    CUtensorMap mQ, mK, mV, mO;
+    if (!map_input(&mQ, Q, p, 128) || !map_input(&mK, K, p, 256) || !map_input(&mV, V, p, 64) ||
+        !map_output(&mO, O, p))
         return RSA_ERR_CUDA;
     for (long long g = 0; g < p.ngroups; ++g) {
         const Group G = group_of(p, g);
         SlabArgs a = slab_args(p, G, dev->status);
-        const uint64_t pitch = uint64_t(p.Lp) * 4;  // fp32 row; P (bf16) in its first half
+        const uint64_t pitch = uint64_t(p.Lp) * 4;  // fp32 row of the slab
         a.nCT = (p.Lp + 255) / 256;
         a.nStat = 2 * a.nCT;
         a.stats = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(slab) +
                                              align_up(size_t(G.nh) * G.R * pitch, kAlign));
-        CUtensorMap mS, mP;
+        CUtensorMap mS, mSld;
         if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
                    pitch * G.R, 32, 32) ||
-            !map3d(&mP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, slab, p.Lp, G.R, G.nh, pitch,
-                   pitch * G.R, 64, 128))
+            !map3d(&mSld, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
+                   pitch * G.R, 32, 128))
             return RSA_ERR_CUDA;
-        // ring pass 1: score slab
+        // ring pass 1: score slab and per-row softmax partials
         a.ntiles = G.nh * a.nRT * a.nCT;
         RSA_LAUNCH(K_QK_SLAB, rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
-        // row softmax over the full key length (partials from the slab GEMM, one streaming pass)
-        RSA_LAUNCH(K_SOFTMAX, rsa::launch_slab_softmax_stream(slab, lse, a, s));
-        // ring pass 2: O = P V
-        a.nCT = 0;
+        // row softmax over the full key length and ring pass 2, O = P V
         a.ntiles = G.nh * a.nRT;
-        a.scale = 1.f;
-        RSA_LAUNCH(K_PV, rsa::launch_ring_rows(mP, mV, O, a, dev->sms, s));
+        RSA_LAUNCH(K_PV, rsa::launch_pv_softmax(mSld, mV, mO, lse, a, dev->sms, s));
     }
     return RSA_OK;
 }

@@ -54,9 +54,11 @@ struct SlabArgs {
 // Each returns a cudaError_t of its launch.
 cudaError_t launch_qk_slab(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mS,
                            const SlabArgs &a, int num_sms, cudaStream_t st);
-// O = P V from the row-major bf16 P slab (mA, 128 x 64 boxes) and V (mB, 64 x 64 boxes).
-cudaError_t launch_ring_rows(const CUtensorMap &mA, const CUtensorMap &mB, void *out,
-                             const SlabArgs &a, int num_sms, cudaStream_t st);
+// Row softmax and ring pass 2: P = 2^(S - m) / l from the fp32 slab (mS: 32 x 128 boxes,
+// 128-byte swizzle) and the partials in a.stats, O = P V (mV: 64 x 64 boxes; mO: [BH][L][d]
+// bf16, 32 x 32 boxes, 64-byte swizzle, store); writes lse of the group's rows.
+cudaError_t launch_pv_softmax(const CUtensorMap &mS, const CUtensorMap &mV, const CUtensorMap &mO,
+                              float *lse, const SlabArgs &a, int num_sms, cudaStream_t st);
 // Key-major backward: recompute P^T, dP^T -> dS^T in TMEM, and dV = P^T dO, dK = scale dS^T Q
 // accumulated in TMEM over the group's query blocks.
 // mStat: the padded row statistics [2][BH][Lp] fp32 (lse * log2(e), then D), box 64 x 1 x 1.
@@ -84,9 +86,6 @@ cudaError_t bwd_kernels_configure();
 // scores, statistics computed here (the fp32 path).
 cudaError_t launch_slab_softmax(float *slab, float *lse, const SlabArgs &a, int p_bf16,
                                 cudaStream_t st);
-// Row softmax of the bf16 path: scores in base-2 units with per-row partials (a.stats) from
-// the slab GEMM; one streaming pass writes bf16 P in place and lse.
-cudaError_t launch_slab_softmax_stream(float *slab, float *lse, const SlabArgs &a, cudaStream_t st);
 // D_i = dO_i . O_i (and lse2 = lse * log2(e) when lse2 != NULL) for all rows of all heads,
 // written in rows padded to Lp with zeros past L.
 cudaError_t launch_rowdot(const void *dO, const void *O, const float *lse, float *Dp,

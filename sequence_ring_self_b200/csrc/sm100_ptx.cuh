@@ -60,27 +60,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// As mbar_try_wait, but the thread may sleep (woken when the phase completes) for up to
-// `hint_ns` before the answer is false, instead of spinning on the issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return done != 0;
-}
-
 // Wait until the phase with the given parity of `bar` has completed. Returns false (and
 // raises *abort) if the CTA was aborted or the wait ran past kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    // plain try_wait polls (each may block for a short, hardware-chosen time): measured a
+    // little faster than asking for long suspends, which wake late
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if ((it & 7u) == 0u) {
             if (*abort) return false;
             if (global_timer_ns() - t0 > kWaitLimitNs) {
