@@ -244,19 +244,11 @@ __device__ __forceinline__ void pdl_trigger() {
 //   K-major:  8 rows x 128 B per atom; SBO = byte distance between 8-row groups.
 //   MN-major: 64 MN-elements (128 B) x 8 K-rows per atom; LBO = byte distance between
 //             64-wide MN blocks, SBO = byte distance between 8-K-row groups.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    d |= static_cast<uint64_t>(2) << 61;
-    return d;
-}
-
-// The same descriptor split into a compile-time constant part (LBO, SBO, version, layout) and
-// the start address field, so that issuing threads only add (address >> 4) per MMA. Shared
-// addresses of a CTA are below 2^18, so the 14-bit start field never carries.
+// The descriptor is split into a compile-time constant part (LBO >> 4 at bits 16..29,
+// SBO >> 4 at bits 32..45, version 1 at bit 46, layout 2 = 128-byte swizzle at bits 61..63)
+// and the start address field (address >> 4, bits 0..13), so that issuing threads only add
+// (address >> 4) per MMA. Shared addresses of a CTA are below 2^18, so the 14-bit start field
+// never carries.
 __host__ __device__ constexpr uint64_t sdesc_const(uint32_t lbo, uint32_t sbo) {
     return (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46) |

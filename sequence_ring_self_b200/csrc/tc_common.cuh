@@ -74,19 +74,7 @@ __device__ __forceinline__ int ring_block(int first, int t, int count) {
     return b >= count ? b - count : b;
 }
 
-// Store 8 packed bf16 values (16 bytes) to global memory.
-__device__ __forceinline__ void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
-                 "r"(d)
-                 : "memory");
-}
 
-
-// Named barrier over `count` threads (count a multiple of 32; ids 1..15, 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // 2^x on the MUFU unit (ex2.approx.ftz: relative error about 2^-22, flushes denormals).
 __device__ __forceinline__ float fast_exp2(float x) {
