@@ -26,7 +26,7 @@ using namespace tc;
 // ======================================================================================
 // qk_slab: S[h][i - r0][j] = log2(e) * scale * Q_i . K_j  (fp32 scores in base-2 units;
 // -inf where j >= L or causal j > i), and per row and 128-column half tile the softmax
-// partials (max_j S, sum_j 2^(S - max)) for the streaming softmax.
+// partials (max_j S, sum_j 2^(S - max)) that pv_softmax combines into each row's statistics.
 // Tile = 128 query rows x 256 keys; K-loop over d in blocks of 64 (one 128-byte swizzle row).
 // 320 threads: producer, MMA, and 8 epilogue warps (2 per TMEM lane quarter, 128 columns each).
 // ======================================================================================

@@ -108,8 +108,8 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
         p.total = fixed;
         return p;
     }
-    // forward: fp32 scores with P written in place (4 B per score); backward (fp32 path):
-    // fp32 P and dS (8 B)
+    // forward: fp32 scores (4 B per score; the fp32 path writes P over them); backward (fp32
+    // path): fp32 P and dS (8 B)
     p.row_bytes = bwd ? size_t(8) * p.Lp : size_t(4) * p.Lp;
     // forward (bf16): plus the per-row softmax partials, one float2 per 128 columns
     if (!bwd && dt == RSA_BF16) p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
