@@ -80,6 +80,9 @@ def kernel_model(w):
     row = BH * L * 4    # one fp32 per row (lse, D)
     return {
         "qk_slab": (2 * p * d, 4 * p + 2 * t),                 # S fp32 write; Q, K read
+        # slab-free forward: pass 1 (S recomputed, not counted; Q K read, lse write), pass 2
+        "fwd_stats": (0, 2 * t + row),
+        "fwd_pv": (2 * p * d, 4 * t + row),                   # Q K V read, O write, lse read
         "pv_softmax": (2 * p * d, 4 * p + 2 * t + row),         # S read, V read, O, lse write
         # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO O K V read,
         # dQ write, lse read, the rows' lse*log2(e) and D written
@@ -275,7 +278,10 @@ def run_gpu(args, w):
     flush = torch.empty(max(1, args.flush_mib) << 20, dtype=torch.uint8, device=dev)
 
     def step():
-        rsa.forward(q, k, v, N, causal, workspace=ws_f, out=o, lse=lse)
+        if args.forward == "recompute":
+            rsa.forward_recompute(q, k, v, N, causal, out=o, lse=lse)
+        else:
+            rsa.forward(q, k, v, N, causal, workspace=ws_f, out=o, lse=lse)
         rsa.backward(q, k, v, o, do, lse, N, causal, workspace=ws_b, dq=dq, dk=dk, dv=dv)
 
     # warm-up; measure how long the host takes to enqueue one step
@@ -338,7 +344,7 @@ def run_gpu(args, w):
     if not args.no_e2e:
         hq, hk, hv, hdo = (x.torch(n).pin_memory() for n in ("q", "k", "v", "do"))
         res = rsa.forward_backward_host(hq, hk, hv, hdo, N, causal, ws_budget=args.ws_budget,
-                                        device=dev)
+                                        device=dev, recompute=args.forward == "recompute")
         torch.cuda.synchronize()
         e_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         e_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -348,7 +354,8 @@ def run_gpu(args, w):
             flush.zero_()
             e_s[i].record()
             rsa.forward_backward_host(hq, hk, hv, hdo, N, causal, ws_budget=args.ws_budget,
-                                      device=dev, results=res)
+                                      device=dev, results=res,
+                                      recompute=args.forward == "recompute")
             e_e[i].record()
         torch.cuda.synchronize()
         dist.barrier()
@@ -415,6 +422,7 @@ def run_gpu(args, w):
                    "head_dim": d, "chunks": N, "causal": causal,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": f"flushed between steps ({args.flush_mib} MiB write)",
+                   "forward": args.forward,
                    "slab_groups": {"forward": plan_f["groups"], "backward": plan_b["groups"],
                                    "workspace_bytes": [nf, nb]}},
         "tokens_per_s": tokens_s,
@@ -487,6 +495,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["sweep"], default="bert")
+    ap.add_argument("--forward", choices=["slab", "recompute"], default="slab",
+                    help="slab: the method's forward (score slab in HBM, the headline path); "
+                         "recompute: the slab-free two-pass forward")
     ap.add_argument("--sweep-L", default="1024,2048,4096,8192,16384,32768")
     ap.add_argument("--sweep-N", default="1,2,4,8,16")
     ap.add_argument("--ws-budget", type=int, default=0, help="workspace budget in bytes (0: default)")

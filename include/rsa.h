@@ -89,6 +89,21 @@ RSA_API rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, vo
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Slab-free forward: the same result as rsa_forward for bf16 (up to the rounding of P), without
+ * a score slab. Pass 1 visits the ring's key blocks for every 128-row tile and keeps only each
+ * row's running max and sum of exponentials (lse); pass 2 recomputes the score tiles on the
+ * chip, forms P = exp(S - lse) there and accumulates O = P V. The recomputation follows the
+ * pages' recomputation in the backward pass (second page, gradient checkpointing), applied to
+ * the forward's two ring passes; the pages themselves keep the scores between the passes.
+ * In:  Q, K, V [B,H,L,d] device bf16 (RSA_BF16 only; RSA_F32 gives RSA_ERR_UNSUPPORTED).
+ * Out: O [B,H,L,d] bf16, lse [B,H,L] fp32 (as rsa_forward's, usable by rsa_backward).
+ * No workspace: nothing but the inputs and outputs lives in device memory.
+ */
+RSA_API rsa_status_t rsa_forward_recompute(const void *Q, const void *K, const void *V, void *O,
+                                           float *lse, int B, int H, int L, int d, int N,
+                                           int causal, rsa_dtype_t dt, void *stream);
+
+/*
  * Backward pass on the same ring schedule: recomputes P from Q, K and lse, forms
  * dP = dO V^T and dS = P * (dP - D) with D_i = dO_i . O_i, then
  * dV_m = sum_n P_n[:, block m]^T dO_n, dK_m = scale sum_n dS_n[:, block m]^T Q_n and

@@ -202,7 +202,8 @@ rsa_status_t device_state(DeviceState **out) {
         e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
         if ((e = rsa::tc_kernels_configure()) != cudaSuccess ||
-            (e = rsa::bwd_kernels_configure()) != cudaSuccess)
+            (e = rsa::bwd_kernels_configure()) != cudaSuccess ||
+            (e = rsa::fwd_kernels_configure()) != cudaSuccess)
             return cuda_fail("cudaFuncSetAttribute", e);
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, rsa::g_status_word);
@@ -227,11 +228,12 @@ rsa_status_t device_state(DeviceState **out) {
 
 enum Kind {
     K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_BWD_ROWS,
-    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_COUNT
+    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_FWD_STATS, K_FWD_PV, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
     "qk_slab", "slab_softmax", "pv_softmax", "rowdot", "bwd_keys", "bwd_rows",
-    "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows"};
+    "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows",
+    "fwd_stats", "fwd_pv"};
 
 struct ProfRec {
     int kind;
@@ -487,6 +489,35 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
         a.ntiles = G.nh * a.nRT;
         RSA_LAUNCH(K_PV, rsa::launch_pv_softmax(mSld, mV, mO, lse, a, dev->sms, s));
     }
+    return RSA_OK;
+}
+
+rsa_status_t rsa_forward_recompute(const void *Q, const void *K, const void *V, void *O,
+                                   float *lse, int B, int H, int L, int d, int N, int causal,
+                                   rsa_dtype_t dt, void *stream) {
+    rsa_status_t why;
+    if (!args_ok(B, H, L, d, N, dt, &why)) return why;
+    if (dt != RSA_BF16) return RSA_ERR_UNSUPPORTED;
+    if (!Q || !K || !V || !O || !lse) return RSA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(lse))
+        return RSA_ERR_INVALID_ARG;
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // one group of every head and row: nothing but Q, K, V, O and lse lives in HBM
+    const Plan p = make_plan(B, H, L, d, N, causal, dt, 1, 0);
+    const uint32_t kn = d == 64 ? 128 : 64;  // keys per step
+    CUtensorMap mQ, mK, mV, mO;
+    if (!map_input(&mQ, Q, p, 128) || !map_input(&mK, K, p, kn) || !map_input(&mV, V, p, kn) ||
+        !map_output(&mO, O, p))
+        return RSA_ERR_CUDA;
+    SlabArgs a = slab_args(p, group_of(p, 0), dev->status);
+    a.ntiles = static_cast<int>(p.BH) * ((L + 127) / 128);
+    // pass 1: per-row max and sum over the ring -> lse
+    RSA_LAUNCH(K_FWD_STATS, rsa::launch_fwd_stats(mQ, mK, lse, a, dev->sms, s));
+    // pass 2: S again, P = 2^(S log2(e) scale - lse log2(e)) on the chip, O = P V
+    RSA_LAUNCH(K_FWD_PV, rsa::launch_fwd_pv(mQ, mK, mV, mO, lse, a, dev->sms, s));
     return RSA_OK;
 }
 

@@ -77,6 +77,16 @@ cudaError_t launch_bwd_rows(const CUtensorMap &mQ, const CUtensorMap &mdO, const
                             const CUtensorMap &mK, const CUtensorMap &mV, const CUtensorMap &mdQ,
                             const float *lse, float *lse2_out, float *d_out, const SlabArgs &a,
                             int num_sms, cudaStream_t st);
+// Slab-free two-pass forward (kernels_fwd.cu), whole problem in one launch each, units of
+// 128 query rows: pass 1 writes lse; pass 2 recomputes S, forms P on the chip and writes O.
+// mQ: 64 x 128 boxes; mK/mV: 64 x KN boxes (KN = 128 keys for d = 64, 64 for d = 128);
+// mO: as for launch_pv_softmax.
+cudaError_t launch_fwd_stats(const CUtensorMap &mQ, const CUtensorMap &mK, float *lse,
+                             const SlabArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_fwd_pv(const CUtensorMap &mQ, const CUtensorMap &mK, const CUtensorMap &mV,
+                          const CUtensorMap &mO, const float *lse, const SlabArgs &a, int num_sms,
+                          cudaStream_t st);
+cudaError_t fwd_kernels_configure();
 cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
 cudaError_t bwd_kernels_configure();
 

@@ -27,7 +27,7 @@ RSA_F32, RSA_BF16 = 0, 1
 EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
             "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
-            "rsa_forward_noalloc", "rsa_last_error")
+            "rsa_forward_noalloc", "rsa_last_error", "rsa_forward_recompute")
 
 _lib = None
 _lock = threading.Lock()
@@ -82,6 +82,8 @@ def load_library(path: str | None = None):
         lib.rsa_profile_read.restype = i
         lib.rsa_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.rsa_forward_noalloc.restype = i
+        lib.rsa_forward_recompute.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+        lib.rsa_forward_recompute.restype = i
         if path is None:
             _lib = lib
         return lib
@@ -194,6 +196,23 @@ def forward(q, k, v, N: int, causal: bool = False, *, ws_budget: int = 0, worksp
     return o, ls
 
 
+def forward_recompute(q, k, v, N: int, causal: bool = False, *, out=None, lse=None,
+                      stream: torch.cuda.Stream | None = None):
+    """Slab-free two-pass forward (bf16): returns (O, lse) like ``forward`` without a workspace."""
+    _check_qkv(q, k, v)
+    B, H, L, d = q.shape
+    dt = _dtype_code(q.dtype)
+    lib = load_library()
+    o = torch.empty_like(q) if out is None else out
+    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib.rsa_forward_recompute(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
+                                   int(bool(causal)), dt, ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_forward_recompute")
+    return o, ls
+
+
 def backward(q, k, v, o, do, lse, N: int, causal: bool = False, *, ws_budget: int = 0,
              workspace=None, dq=None, dk=None, dv=None, stream: torch.cuda.Stream | None = None):
     """Ring Self-Attention backward. Returns (dQ, dK, dV) in the input dtype."""
@@ -256,13 +275,17 @@ class RingSelfAttention(torch.autograd.Function):
 
 
 def forward_backward_host(q, k, v, do, N: int, causal: bool = False, *, ws_budget: int = 0,
-                          device=None, results=None):
+                          device=None, results=None, recompute: bool = False):
     """One forward + backward from host (ideally pinned) tensors: copies Q, K, V, dO to the
     device, runs the library's forward and backward there, and copies O, lse, dQ, dK, dV
-    back into host tensors (``results`` if given, a dict of pinned tensors by name)."""
+    back into host tensors (``results`` if given, a dict of pinned tensors by name).
+    ``recompute`` selects the slab-free forward."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in (q, k, v, do))
-    o, lse = forward(qd, kd, vd, N, causal, ws_budget=ws_budget)
+    if recompute:
+        o, lse = forward_recompute(qd, kd, vd, N, causal)
+    else:
+        o, lse = forward(qd, kd, vd, N, causal, ws_budget=ws_budget)
     dq, dk, dv = backward(qd, kd, vd, o, dod, lse, N, causal, ws_budget=ws_budget)
     names = ("O", "lse", "dQ", "dK", "dV")
     if results is None:

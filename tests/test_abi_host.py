@@ -76,6 +76,20 @@ def test_cuda_failures_are_described(lib):
         raise rsa.RSAError(rsa.RSA_ERR_CUDA, "rsa_backward")
 
 
+def _fwdr(lib, B=1, H=1, L=128, d=64, N=1, dt=rsa.RSA_BF16, ptr=FAKE, lse=FAKE):
+    return lib.rsa_forward_recompute(ptr, ptr, ptr, ptr, lse, B, H, L, d, N, 0, dt, None)
+
+
+def test_forward_recompute_argument_errors(lib):
+    assert _fwdr(lib, L=100, N=3) == rsa.RSA_ERR_INVALID_ARG
+    assert _fwdr(lib, B=0) == rsa.RSA_ERR_INVALID_ARG
+    assert _fwdr(lib, d=96) == rsa.RSA_ERR_UNSUPPORTED
+    assert _fwdr(lib, d=64, dt=rsa.RSA_F32) == rsa.RSA_ERR_UNSUPPORTED  # bf16 only
+    assert _fwdr(lib, ptr=0) == rsa.RSA_ERR_INVALID_ARG
+    assert _fwdr(lib, lse=0) == rsa.RSA_ERR_INVALID_ARG
+    assert _fwdr(lib, ptr=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG
+
+
 def test_forward_rejects_null_lse(lib):
     assert _fwd(lib, lse=0) == rsa.RSA_ERR_INVALID_ARG
 

@@ -296,6 +296,47 @@ def test_autograd_wrapper_and_host_api(orc):
         np.testing.assert_array_equal(res[n].to(torch.float64).numpy(), ref[n])
 
 
+RECOMPUTE_SHAPES = [  # (B, H, L, d, N, causal)
+    (2, 3, 512, 64, 4, False),
+    (2, 3, 512, 64, 4, True),
+    (1, 3, 200, 128, 4, False),  # d = 128, ragged
+    (1, 2, 700, 128, 7, True),
+    (1, 1, 1, 64, 1, False),     # one token
+    (1, 2, 50, 64, 5, True),     # smaller than one tile
+    (2, 1, 130, 64, 2, True),    # one tile plus a 2-row tail
+]
+
+
+@pytest.mark.parametrize("shape", RECOMPUTE_SHAPES)
+def test_forward_recompute_matches_oracle_and_slab_forward(orc, shape):
+    """The slab-free two-pass forward: O and lse against the oracle, and against the slab
+    forward within the bf16 bound; its lse drives the backward like the slab forward's."""
+    B, H, L, d, N, causal = shape
+    x = make_inputs(B, H, L, d, seed=600 + L + d + int(causal), dtype="bf16")
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+    o, lse = rsa.forward_recompute(q, k, v, N, causal)
+    dq, dk, dv = rsa.backward(q, k, v, o, do, lse, N, causal)
+    torch.cuda.synchronize()
+    assert rsa.last_device_status() == rsa.RSA_OK
+    o_ref, lse_ref = orc.forward(x.q, x.k, x.v, causal)
+    check(np64(o), o_ref, "bf16", "O (recompute)")
+    np.testing.assert_allclose(np64(lse), lse_ref, rtol=0, atol=1e-3)
+    slab = run(x, N, causal, bwd=False)
+    check(np64(o), slab["O"], "bf16", "O recompute vs slab")
+    np.testing.assert_allclose(np64(lse), slab["lse"], rtol=0, atol=1e-5)
+    for name, ref, got in zip(("dQ", "dK", "dV"), orc.backward(x.q, x.k, x.v, x.do, causal),
+                              (dq, dk, dv)):
+        check(np64(got), ref, "bf16", f"{name} after the recompute forward")
+
+
+def test_forward_recompute_rejects_fp32():
+    q = torch.zeros(1, 1, 64, 32, dtype=torch.float32, device=torch.device("cuda", 0))
+    with pytest.raises(rsa.RSAError) as e:
+        rsa.forward_recompute(q, q, q, 1)
+    assert e.value.code == rsa.RSA_ERR_UNSUPPORTED
+
+
 def test_calls_from_a_fresh_thread():
     """A thread that has made no CUDA call yet (as autograd's backward thread may be) can call
     the library: it binds the device's context itself before encoding its tensor maps."""
