@@ -23,7 +23,8 @@
  *   - scale = 1/sqrt(d) is fixed. causal != 0 keeps keys j <= i only (the diagonal is kept).
  *     No dropout, bias or padding mask.
  *   - Supported: B, H, L >= 1, N >= 1 with L % N == 0; bf16 with d in {64, 128}; fp32 with
- *     d in {32, 64}. L need not be a multiple of any tile size.
+ *     d in {32, 64}; L <= 2^22 and B * H * ceil(L / 128) < 2^30. L need not be a multiple of
+ *     any tile size.
  *   - Arithmetic: bf16 inputs with fp32 accumulation and fp32 softmax statistics; P and dS
  *     are rounded to bf16 before their GEMMs; outputs are rounded to nearest-even into `dt`.
  *     The fp32 path computes every step in fp32 on the CUDA cores (no TF32).
@@ -51,7 +52,7 @@ extern "C" {
 typedef enum {
     RSA_OK = 0,
     RSA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, L % N != 0 */
-    RSA_ERR_UNSUPPORTED = 2, /* head dim or dtype outside the supported set, no sm_100 GPU */
+    RSA_ERR_UNSUPPORTED = 2, /* head dim, dtype or size outside the supported set, no sm_100 GPU */
     RSA_ERR_WORKSPACE = 3,   /* workspace smaller than the minimum plan needs */
     RSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
     RSA_ERR_TIMEOUT = 5      /* a kernel's bounded wait ran out (reported afterwards) */

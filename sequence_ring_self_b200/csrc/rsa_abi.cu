@@ -64,7 +64,9 @@ bool args_ok(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *wh
         *why = RSA_ERR_INVALID_ARG;
         return false;
     }
-    if (L > (1 << 22) || static_cast<long long>(B) * H > 0x7fffffffLL) {
+    // work units (B*H heads x 128-row tiles) are counted in 32-bit ints by the kernels
+    const long long BH = static_cast<long long>(B) * H;
+    if (L > (1 << 22) || BH > 0x7fffffffLL || BH * ((L + 127) / 128) > 0x3fffffffLL) {
         *why = RSA_ERR_UNSUPPORTED;
         return false;
     }

@@ -90,6 +90,14 @@ def test_forward_recompute_argument_errors(lib):
     assert _fwdr(lib, ptr=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG
 
 
+def test_sizes_beyond_the_unit_counters_are_unsupported(lib):
+    # 2^24 heads of 2^16 rows: more 128-row units than a 32-bit counter holds
+    assert lib.rsa_workspace_size(1 << 12, 1 << 12, 1 << 16, 64, 1, 0, rsa.RSA_BF16, 0, 0) == 0
+    assert _fwd(lib, B=1 << 12, H=1 << 12, L=1 << 16) == rsa.RSA_ERR_UNSUPPORTED
+    assert _bwd(lib, B=1 << 12, H=1 << 12, L=1 << 16) == rsa.RSA_ERR_UNSUPPORTED
+    assert _fwdr(lib, B=1 << 12, H=1 << 12, L=1 << 16) == rsa.RSA_ERR_UNSUPPORTED
+
+
 def test_forward_rejects_null_lse(lib):
     assert _fwd(lib, lse=0) == rsa.RSA_ERR_INVALID_ARG
 
