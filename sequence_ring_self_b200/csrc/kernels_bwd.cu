@@ -15,15 +15,17 @@
 // the manner of recomputation in the backward pass. The epilogue writes P^T and dS^T as bf16
 // pairs back into the TMEM columns it has just read S^T and dP^T from, and the dV/dK MMAs take
 // their A operand from there. dQ comes from the row-major companion kernel below, which
-// recomputes S, P, dP and dS for its query rows, so no dS slab is ever written.
+// recomputes S, P, dP and dS for its query rows, so no dS slab is ever written; it runs first
+// and also writes the rows' statistics (lse log2(e) and D_i = dO_i . O_i) this kernel reads.
 //
 // Roles (320 threads): warp 0 lane 0 issues TMA loads (K/V per key tile, Q/dO and the rows'
 // statistics per step); warp 1 owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the
 // epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (keys) and query columns 32*((w-2)/4)..+31.
-// The S^T/dP^T accumulators are double-buffered and the MMA warp issues step t's S^T/dP^T
-// before step t-1's dV/dK, so the tensor core works on one step while the epilogue works on
-// the previous one. MMAs of one thread execute in issue order, so step t's dV/dK MMAs read
-// P^T/dS^T of buffer b before step t+2's S^T/dP^T MMAs overwrite it.
+// The S^T/dP^T accumulators are double-buffered and the MMA warp issues a step's S^T/dP^T
+// ahead of the previous step's dV/dK (two steps ahead for d = 64, one for d = 128), so the
+// tensor core works on one step while the epilogue works on another. MMAs of one thread
+// execute in issue order, so step t's dV/dK MMAs read P^T/dS^T of buffer b before step t+2's
+// S^T/dP^T MMAs overwrite it.
 #include "tc_common.cuh"
 
 namespace rsa {
