@@ -80,9 +80,10 @@ def kernel_model(w):
     row = BH * L * 4    # one fp32 per row (lse, D)
     return {
         "qk_slab": (2 * p * d, 4 * p + 2 * t),                 # S fp32 write; Q, K read
-        # slab-free forward: pass 1 (S recomputed, not counted; Q K read, lse write), pass 2
-        "fwd_stats": (0, 2 * t + row),
-        "fwd_pv": (2 * p * d, 4 * t + row),                   # Q K V read, O write, lse read
+        # slab-free forward: pass 1 (QK^T; Q K read, lse write), pass 2 (PV, with S recomputed,
+        # not counted; Q K V read, O write, lse read)
+        "fwd_stats": (2 * p * d, 2 * t + row),
+        "fwd_pv": (2 * p * d, 4 * t + row),
         "pv_softmax": (2 * p * d, 4 * p + 2 * t + row),         # S read, V read, O, lse write
         # query-major backward: dQ (+ the recomputed S and dP, not counted); Q dO O K V read,
         # dQ write, lse read, the rows' lse*log2(e) and D written
