@@ -29,8 +29,12 @@
  *     are rounded to bf16 before their GEMMs; outputs are rounded to nearest-even into `dt`.
  *     The fp32 path computes every step in fp32 on the CUDA cores (no TF32).
  *   - Ownership: the caller owns every buffer, including `workspace`. The library never
- *     allocates or frees device memory and never synchronises `stream` (a cudaStream_t;
- *     NULL means the legacy default stream). Work is enqueued on `stream` in order.
+ *     allocates or frees device memory at run time and never synchronises `stream` (a
+ *     cudaStream_t; NULL means the legacy default stream). Work is enqueued on `stream` in
+ *     order. The one piece of device memory the library holds itself is the fixed scratch
+ *     array of rsa_forward_noalloc (see there), a static part of the library's device code.
+ *   - Device: calls run on the calling thread's current CUDA device. Every pointer passed and
+ *     `stream` must belong to that device; make it current (cudaSetDevice) first.
  *   - Errors: arguments are checked before anything is launched; a failed check returns an
  *     error code and enqueues nothing. Nothing throws across this interface.
  */
@@ -64,10 +68,13 @@ typedef enum { RSA_F32 = 0, RSA_BF16 = 1 } rsa_dtype_t;
  * Bytes of device workspace a call needs.
  *
  * The score slab (the c x L block of scores of every chunk, i.e. L x L per head) is
- * processed in groups: a group is a set of whole heads, or, when one head does not fit, a
- * range of rows (a multiple of 128) of one head. `budget_bytes` caps the workspace: the
- * returned size is that of the largest plan that fits the budget (or of the smallest plan if
- * none fits). budget_bytes == 0 asks for the default plan (at most 1 GiB).
+ * processed in groups, one after the other in the same workspace: a group is a set of whole
+ * heads, or, when a head does not fit, the same range of rows (a multiple of 128) of one or
+ * several heads. On the bf16 forward the groups are balanced: equal rectangles of heads x rows
+ * chosen so that no group is a small remainder that would leave most of the GPU idle.
+ * `budget_bytes` caps the workspace: the returned size is that of the plan chosen within the
+ * budget (or of the smallest plan, one 128-row range of one head, if nothing fits).
+ * budget_bytes == 0 asks for the default plan (at most 1 GiB).
  * for_backward selects the backward call's needs: on the bf16 path the backward keeps no
  * slab (every score tile is recomputed on the chip) and needs only the padded per-row
  * statistics, 8 * B * H * roundup(L, 64) bytes, whatever the budget; the fp32 path keeps fp32
@@ -139,6 +146,15 @@ RSA_API const char *rsa_last_error(void);
 RSA_API rsa_status_t rsa_last_device_status(void *stream);
 
 /*
+ * Posts `code` (RSA_OK or RSA_ERR_TIMEOUT) into the current device's status word from a
+ * one-thread kernel on `stream`, exactly as a kernel whose bounded wait gave up records its
+ * failure. A failure-injection hook for testing the reporting path (rsa_last_device_status
+ * must then return the code and clear it) without making any wait run out. Not part of the
+ * paper's method. RSA_ERR_INVALID_ARG for any other code.
+ */
+RSA_API rsa_status_t rsa_debug_report_status(int code, void *stream);
+
+/*
  * The plan a call with these arguments and ws_bytes would use, for inspection:
  * out[0] = number of groups, out[1] = heads per group, out[2] = rows per group,
  * out[3] = padded row length of the slab (elements), out[4] = bytes the plan uses.
@@ -161,6 +177,18 @@ RSA_API int rsa_profile_kinds(void);
 RSA_API const char *rsa_profile_kind_name(int kind); /* NULL if out of range */
 RSA_API rsa_status_t rsa_profile_read(double *ms, long long *launches);
 
+/*
+ * FP32 FMA throughput probe (a benchmark helper, not part of the method): the denominator of
+ * the fp32 path's roofline, which runs on the CUDA cores. Launches `blocks` blocks of 256
+ * threads on `stream`; every thread performs rsa_probe_ffma_flops_per_thread(iters) flops of
+ * independent FMA chains. The caller times the launch (CUDA events on `stream`) and divides.
+ * out: device buffer of at least `blocks` floats (written only in a case that never occurs,
+ * so that the compiler keeps the work). Returns RSA_ERR_INVALID_ARG for a NULL buffer or
+ * non-positive counts, RSA_ERR_CUDA if the launch fails.
+ */
+RSA_API rsa_status_t rsa_probe_ffma(void *out, int blocks, int iters, void *stream);
+RSA_API long long rsa_probe_ffma_flops_per_thread(int iters);
+
 /* Size of the scratch array rsa_forward_noalloc works in: 32 MiB of device memory per GPU
  * that loads the library, held until the process exits. */
 #define RSA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -176,8 +204,15 @@ RSA_API rsa_status_t rsa_profile_read(double *ms, long long *launches);
  * calls no allocating routine.
  * - Problems whose smallest plan does not fit the scratch (rows longer than about 64,000
  *   keys) are rejected with RSA_ERR_WORKSPACE before anything is launched.
- * - The first call on a device looks up the scratch array's device address on that device;
- *   make that first call before any stream capture on the device.
+ * - The scratch array is part of the library's device code, so it occupies device memory
+ *   once the code module holding it is loaded on a device: under CUDA's default lazy module
+ *   loading that happens at the first rsa_forward_noalloc call on the device (whose address
+ *   lookup loads the module), with CUDA_MODULE_LOADING=EAGER when the library's context is
+ *   created. It stays until the process exits.
+ * - The first call on a device looks up the scratch array's device address on that device,
+ *   after the same argument and device checks rsa_forward makes (so both entry points return
+ *   the same codes for the same arguments); make that first call before any stream capture
+ *   on the device.
  * - Every call on a device uses the same scratch array, and it keeps the last call's
  *   contents (nothing in it needs to start cleared: each call writes every byte it reads).
  *   Calls whose work overlaps on the GPU (for example on two streams without ordering

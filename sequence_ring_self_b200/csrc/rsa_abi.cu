@@ -50,9 +50,10 @@ struct Plan {
     rsa_dtype_t dt;
     long long BH;
     int Lp, c;
-    int whole;     // groups of whole heads
-    long long Gh;  // heads per group (whole mode)
-    int R;         // rows per group (row mode); L in whole mode
+    int whole;     // every group holds whole heads (R == L)
+    long long Gh;  // heads per group
+    int R;         // rows per group (a multiple of 128, or L)
+    long long gt;  // row groups per head: ceil(L / R)
     long long ngroups;
     size_t row_bytes;   // slab bytes per row (all slabs of the pass)
     size_t slab_bytes;  // slab region
@@ -87,6 +88,60 @@ bool args_ok(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *wh
     return true;
 }
 
+// Work units a slab group should hold for its two kernels to keep HBM busy: a group with fewer
+// (128-row tile, head) units runs about as long as one with this many, since each unit streams
+// its scores at the rate of one SM.
+constexpr long long kSaturatingUnits = 96;
+
+// bf16 forward: groups are rectangles of Gh heads x R rows (R = rt * 128, or L). Among the
+// rectangles that fit the budget, take the one whose groups cost least in total, a group
+// costing max(its units, kSaturatingUnits): equal groups, none of them a small tail that would
+// run as long as a full one. Head counts are enumerated by their distinct balanced values.
+void plan_rect(Plan &p, size_t budget) {
+    const long long nRT = (p.L + 127) / 128;
+    const size_t tile_bytes = size_t(128) * p.row_bytes;  // one 128-row tile of one head
+    const size_t head_bytes = size_t(p.L) * p.row_bytes;
+    const long long fit_tiles = static_cast<long long>(budget / tile_bytes);
+    const long long fit_heads = static_cast<long long>(budget / head_bytes);
+    long long best_cost = -1, best_groups = 0, best_nh = 1, best_rt = 1;
+    for (long long gh = 1; gh <= p.BH;) {
+        const long long nh = (p.BH + gh - 1) / gh;  // heads per group with gh head groups
+        long long rt = 0;
+        if (fit_heads >= nh)
+            rt = nRT;
+        else if (fit_tiles >= nh)
+            rt = fit_tiles / nh;
+        if (rt > 0) {
+            const long long ngh = (p.BH + nh - 1) / nh, last_h = p.BH - (ngh - 1) * nh;
+            long long ngt = (nRT + rt - 1) / rt;
+            const long long rt2 = (nRT + ngt - 1) / ngt;  // balanced tile count
+            ngt = (nRT + rt2 - 1) / rt2;
+            const long long last_t = nRT - (ngt - 1) * rt2;
+            auto c = [](long long u) { return u > kSaturatingUnits ? u : kSaturatingUnits; };
+            const long long cost = (ngh - 1) * (ngt - 1) * c(nh * rt2) + (ngh - 1) * c(nh * last_t) +
+                                   (ngt - 1) * c(last_h * rt2) + c(last_h * last_t);
+            const long long groups = ngh * ngt;
+            if (best_cost < 0 || cost < best_cost || (cost == best_cost && groups < best_groups)) {
+                best_cost = cost;
+                best_groups = groups;
+                best_nh = nh;
+                best_rt = rt2;
+            }
+        }
+        if (nh == 1) break;
+        gh = (p.BH + nh - 2) / (nh - 1);  // the next head-group count with fewer heads per group
+    }
+    // nothing fits: the smallest plan (one 128-row tile of one head)
+    p.Gh = best_nh;
+    p.R = best_rt * 128 >= p.L ? p.L : static_cast<int>(best_rt * 128);
+    p.whole = p.R == p.L;
+    p.gt = (p.L + p.R - 1) / p.R;
+    p.ngroups = ((p.BH + p.Gh - 1) / p.Gh) * p.gt;
+    p.slab_bytes = align_up(size_t(p.Gh) * p.R * p.row_bytes, kAlign);
+    p.off_D = p.slab_bytes;
+    p.total = p.off_D;
+}
+
 // Largest plan whose workspace fits `budget` (the smallest plan if none does).
 Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, int bwd,
                size_t budget) {
@@ -96,6 +151,7 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     p.BH = static_cast<long long>(B) * H;
     p.Lp = (L + 63) / 64 * 64;
     p.c = L / N;
+    p.gt = 1;
     // backward: padded row statistics D and lse * log2(e), [2][BH][Lp] fp32
     const size_t fixed = bwd ? align_up(size_t(2) * p.BH * p.Lp * 4, kAlign) : 0;
     if (bwd && dt == RSA_BF16) {
@@ -113,8 +169,12 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     // forward: fp32 scores (4 B per score; the fp32 path writes P over them); backward (fp32
     // path): fp32 P and dS (8 B)
     p.row_bytes = bwd ? size_t(8) * p.Lp : size_t(4) * p.Lp;
-    // forward (bf16): plus the per-row softmax partials, one float2 per 128 columns
-    if (!bwd && dt == RSA_BF16) p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
+    if (!bwd && dt == RSA_BF16) {
+        // plus the per-row softmax partials, one float2 per 128 columns
+        p.row_bytes += size_t(8) * 2 * ((p.Lp + 255) / 256);
+        plan_rect(p, budget);
+        return p;
+    }
     const size_t head_bytes = align_up(size_t(L) * p.row_bytes, kAlign);
     if (budget >= fixed + head_bytes) {
         p.whole = 1;
@@ -142,8 +202,8 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
             return p;
         }
         p.R = static_cast<int>(r);
-        const long long per_head = (L + p.R - 1) / p.R;
-        p.ngroups = p.BH * per_head;
+        p.gt = (L + p.R - 1) / p.R;
+        p.ngroups = p.BH * p.gt;
         p.slab_bytes = align_up(size_t(p.R) * p.row_bytes, kAlign);
         p.off_D = p.slab_bytes;
         p.total = p.off_D + fixed;
@@ -151,25 +211,17 @@ Plan make_plan(int B, int H, int L, int d, int N, int causal, rsa_dtype_t dt, in
     return p;
 }
 
+// Group g of a plan: head group g / gt, row group g % gt.
 Group group_of(const Plan &p, long long g) {
     Group G{};
-    if (p.whole) {
-        G.bh0 = static_cast<int>(g * p.Gh);
-        long long nh = p.BH - g * p.Gh;
-        G.nh = static_cast<int>(nh < p.Gh ? nh : p.Gh);
-        G.r0 = 0;
-        G.R = p.L;
-        G.first_of_head = G.last_of_head = 1;
-    } else {
-        const long long per_head = (p.L + p.R - 1) / p.R;
-        G.bh0 = static_cast<int>(g / per_head);
-        G.nh = 1;
-        const int k = static_cast<int>(g - static_cast<long long>(G.bh0) * per_head);
-        G.r0 = k * p.R;
-        G.R = p.L - G.r0 < p.R ? p.L - G.r0 : p.R;
-        G.first_of_head = k == 0;
-        G.last_of_head = G.r0 + G.R == p.L;
-    }
+    const long long hg = g / p.gt, rg = g - hg * p.gt;
+    G.bh0 = static_cast<int>(hg * p.Gh);
+    const long long nh = p.BH - hg * p.Gh;
+    G.nh = static_cast<int>(nh < p.Gh ? nh : p.Gh);
+    G.r0 = static_cast<int>(rg * p.R);
+    G.R = p.L - G.r0 < p.R ? p.L - G.r0 : p.R;
+    G.first_of_head = G.r0 == 0;
+    G.last_of_head = G.r0 + G.R == p.L;
     return G;
 }
 
@@ -354,7 +406,34 @@ rsa_status_t check_common(const Plan &p, void *ws, size_t ws_bytes) {
 
 }  // namespace
 
+bool rsa::check_args(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *why) {
+    return args_ok(B, H, L, d, N, dt, why);
+}
+
+rsa_status_t rsa::check_device() {
+    DeviceState *s = nullptr;
+    return device_state(&s);
+}
+
+rsa_status_t rsa::record_cuda_failure(const char *what, cudaError_t e) { return cuda_fail(what, e); }
+
+namespace {
+// Writes `code` into the device status word from the GPU, as a kernel whose bounded wait gave
+// up does (see rsa_debug_report_status).
+__global__ void report_status_kernel(int *word, int code) { atomicExch(word, code); }
+}  // namespace
+
 extern "C" {
+
+rsa_status_t rsa_debug_report_status(int code, void *stream) {
+    if (code != RSA_OK && code != RSA_ERR_TIMEOUT) return RSA_ERR_INVALID_ARG;
+    DeviceState *s = nullptr;
+    const rsa_status_t st = device_state(&s);
+    if (st != RSA_OK) return st;
+    report_status_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(s->status, code);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? RSA_OK : cuda_fail("report_status_kernel", e);
+}
 
 const char *rsa_status_string(rsa_status_t s) {
     switch (s) {
@@ -384,7 +463,7 @@ rsa_status_t rsa_plan_describe(int B, int H, int L, int d, int N, int causal, rs
     if (!args_ok(B, H, L, d, N, dt, &why)) return why;
     const Plan p = make_plan(B, H, L, d, N, causal, dt, for_backward, ws_bytes);
     out[0] = p.ngroups;
-    out[1] = p.whole ? p.Gh : 1;
+    out[1] = p.Gh;
     out[2] = p.R;
     out[3] = p.Lp;
     out[4] = static_cast<long long>(p.total);

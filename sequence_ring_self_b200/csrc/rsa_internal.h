@@ -6,7 +6,19 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/rsa.h"
+
 namespace rsa {
+
+// ---- checks shared by the entry points (rsa_abi.cu) --------------------------------------
+// Argument checks of every forward/backward entry point: sizes, divisibility, supported head
+// dimension and dtype. On failure returns false and sets *why.
+bool check_args(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *why);
+// Binds the current device's primary context on the calling thread and checks once per device
+// that it is an sm_100 GPU (RSA_ERR_UNSUPPORTED otherwise); configures the kernels.
+rsa_status_t check_device();
+// Records which CUDA call failed (read back by rsa_last_error) and returns RSA_ERR_CUDA.
+rsa_status_t record_cuda_failure(const char *what, cudaError_t e);
 
 // Launch with programmatic stream serialisation: the kernel may start (and run its prologue)
 // while the previous kernel in the stream finishes; it calls pdl_wait() before touching memory

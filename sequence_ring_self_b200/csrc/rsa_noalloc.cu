@@ -29,12 +29,15 @@ void *g_scratch[kMaxDevices];  // device address of g_noalloc_scratch, per devic
 
 rsa_status_t scratch_of_current_device(void **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return RSA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return rsa::record_cuda_failure("cudaGetDevice", e);
     if (dev < 0 || dev >= kMaxDevices) return RSA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_scratch[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RSA_ERR_CUDA;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return rsa::record_cuda_failure("cudaGetSymbolAddress(scratch)", e);
+        if (!p) return RSA_ERR_CUDA;
         g_scratch[dev] = p;
     }
     *out = g_scratch[dev];
@@ -46,12 +49,21 @@ rsa_status_t scratch_of_current_device(void **out) {
 extern "C" rsa_status_t rsa_forward_noalloc(const void *Q, const void *K, const void *V, void *O,
                                             float *lse, int B, int H, int L, int d, int N,
                                             int causal, rsa_dtype_t dt, void *stream) {
-    // the largest plan that fits the scratch; 0 means the arguments are invalid
+    // the checks rsa_forward makes, in its order, so that both report the same code
+    rsa_status_t st;
+    if (!rsa::check_args(B, H, L, d, N, dt, &st)) return st;
+    if (!Q || !K || !V || !O || !lse) return RSA_ERR_INVALID_ARG;
+    for (const void *p : {static_cast<const void *>(Q), K, V, static_cast<const void *>(O),
+                          static_cast<const void *>(lse)})
+        if (reinterpret_cast<uintptr_t>(p) & 15u) return RSA_ERR_INVALID_ARG;
+    // the largest plan that fits the scratch
     const size_t need = rsa_workspace_size(B, H, L, d, N, causal, dt, 0, kScratchBytes);
-    if (need == 0) return RSA_ERR_INVALID_ARG;
     if (need > kScratchBytes) return RSA_ERR_WORKSPACE;  // even the smallest plan does not fit
+    // an sm_100 device (and its context on this thread) before the scratch lookup
+    st = rsa::check_device();
+    if (st != RSA_OK) return st;
     void *scratch = nullptr;
-    const rsa_status_t st = scratch_of_current_device(&scratch);
+    st = scratch_of_current_device(&scratch);
     if (st != RSA_OK) return st;
     return rsa_forward(Q, K, V, O, lse, B, H, L, d, N, causal, dt, scratch, kScratchBytes, stream);
 }

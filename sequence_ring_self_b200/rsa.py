@@ -27,7 +27,8 @@ RSA_F32, RSA_BF16 = 0, 1
 EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_string",
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
             "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
-            "rsa_forward_noalloc", "rsa_last_error", "rsa_forward_recompute")
+            "rsa_forward_noalloc", "rsa_last_error", "rsa_forward_recompute",
+            "rsa_probe_ffma", "rsa_probe_ffma_flops_per_thread", "rsa_debug_report_status")
 
 _lib = None
 _lock = threading.Lock()
@@ -84,6 +85,12 @@ def load_library(path: str | None = None):
         lib.rsa_forward_noalloc.restype = i
         lib.rsa_forward_recompute.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         lib.rsa_forward_recompute.restype = i
+        lib.rsa_probe_ffma.argtypes = [vp, i, i, vp]
+        lib.rsa_probe_ffma.restype = i
+        lib.rsa_probe_ffma_flops_per_thread.argtypes = [i]
+        lib.rsa_probe_ffma_flops_per_thread.restype = ctypes.c_longlong
+        lib.rsa_debug_report_status.argtypes = [i, vp]
+        lib.rsa_debug_report_status.restype = i
         if path is None:
             _lib = lib
         return lib
@@ -123,8 +130,21 @@ def plan_describe(B: int, H: int, L: int, d: int, N: int, causal: bool, dtype: t
 
 
 def last_device_status(stream: torch.cuda.Stream | None = None) -> int:
+    """Status the kernels reported on the stream's device (RSA_OK or RSA_ERR_TIMEOUT) since the
+    last call; synchronises the stream and clears the status."""
     s = stream if stream is not None else torch.cuda.current_stream()
-    return int(load_library().rsa_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+    with torch.cuda.device(s.device):
+        return int(load_library().rsa_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def debug_report_status(code: int, stream: torch.cuda.Stream | None = None) -> None:
+    """Post a status code into the device status word from the GPU, as a kernel whose bounded
+    wait gave up does (a failure-injection hook for testing the reporting path)."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.device(s.device):
+        rc = load_library().rsa_debug_report_status(int(code), ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_debug_report_status")
 
 
 def profile_enable(on: bool) -> None:
@@ -174,23 +194,33 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _same_device(device, *ts):
+    """Outputs and workspaces given by the caller must live on the inputs' device."""
+    for t in ts:
+        if t is not None and t.device != device:
+            raise ValueError(f"tensor on {t.device}, expected {device} (the inputs' device)")
+
+
 def forward(q, k, v, N: int, causal: bool = False, *, ws_budget: int = 0, workspace=None,
             out=None, lse=None, stream: torch.cuda.Stream | None = None):
     """Ring Self-Attention forward. Returns (O [B,H,L,d] in the input dtype, lse [B,H,L] fp32)."""
     _check_qkv(q, k, v)
+    _same_device(q.device, out, lse)
     B, H, L, d = q.shape
     dt = _dtype_code(q.dtype)
     lib = load_library()
     nbytes = lib.rsa_workspace_size(B, H, L, d, N, int(bool(causal)), dt, 0, int(ws_budget))
     if nbytes == 0:
         raise RSAError(RSA_ERR_INVALID_ARG, "rsa_forward")
-    ws = _workspace(nbytes, q.device, workspace)
-    o = torch.empty_like(q) if out is None else out
-    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = lib.rsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
-                         int(bool(causal)), dt, _ptr(ws), ws.numel() * ws.element_size(),
-                         ctypes.c_void_p(s.cuda_stream))
+    # the library runs on the current device: make it the tensors' device for the call
+    with torch.cuda.device(q.device):
+        ws = _workspace(nbytes, q.device, workspace)
+        o = torch.empty_like(q) if out is None else out
+        ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = lib.rsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
+                             int(bool(causal)), dt, _ptr(ws), ws.numel() * ws.element_size(),
+                             ctypes.c_void_p(s.cuda_stream))
     if rc != RSA_OK:
         raise RSAError(rc, "rsa_forward")
     return o, ls
@@ -200,14 +230,16 @@ def forward_recompute(q, k, v, N: int, causal: bool = False, *, out=None, lse=No
                       stream: torch.cuda.Stream | None = None):
     """Slab-free two-pass forward (bf16): returns (O, lse) like ``forward`` without a workspace."""
     _check_qkv(q, k, v)
+    _same_device(q.device, out, lse)
     B, H, L, d = q.shape
     dt = _dtype_code(q.dtype)
     lib = load_library()
-    o = torch.empty_like(q) if out is None else out
-    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = lib.rsa_forward_recompute(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
-                                   int(bool(causal)), dt, ctypes.c_void_p(s.cuda_stream))
+    with torch.cuda.device(q.device):
+        o = torch.empty_like(q) if out is None else out
+        ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = lib.rsa_forward_recompute(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d, N,
+                                       int(bool(causal)), dt, ctypes.c_void_p(s.cuda_stream))
     if rc != RSA_OK:
         raise RSAError(rc, "rsa_forward_recompute")
     return o, ls
@@ -217,6 +249,7 @@ def backward(q, k, v, o, do, lse, N: int, causal: bool = False, *, ws_budget: in
              workspace=None, dq=None, dk=None, dv=None, stream: torch.cuda.Stream | None = None):
     """Ring Self-Attention backward. Returns (dQ, dK, dV) in the input dtype."""
     _check_qkv(q, k, v, o, do)
+    _same_device(q.device, lse, dq, dk, dv)
     B, H, L, d = q.shape
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, L) or not lse.is_contiguous():
         raise ValueError("lse must be contiguous fp32 [B, H, L]")
@@ -225,14 +258,15 @@ def backward(q, k, v, o, do, lse, N: int, causal: bool = False, *, ws_budget: in
     nbytes = lib.rsa_workspace_size(B, H, L, d, N, int(bool(causal)), dt, 1, int(ws_budget))
     if nbytes == 0:
         raise RSAError(RSA_ERR_INVALID_ARG, "rsa_backward")
-    ws = _workspace(nbytes, q.device, workspace)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = lib.rsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
-                          _ptr(dk), _ptr(dv), B, H, L, d, N, int(bool(causal)), dt, _ptr(ws),
-                          ws.numel() * ws.element_size(), ctypes.c_void_p(s.cuda_stream))
+    with torch.cuda.device(q.device):
+        ws = _workspace(nbytes, q.device, workspace)
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(q) if dk is None else dk
+        dv = torch.empty_like(q) if dv is None else dv
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = lib.rsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                              _ptr(dk), _ptr(dv), B, H, L, d, N, int(bool(causal)), dt, _ptr(ws),
+                              ws.numel() * ws.element_size(), ctypes.c_void_p(s.cuda_stream))
     if rc != RSA_OK:
         raise RSAError(rc, "rsa_backward")
     return dq, dk, dv
@@ -245,13 +279,15 @@ def forward_noalloc(q, k, v, N: int, causal: bool = False, *, out=None, lse=None
     memory. Pass `out` and `lse` to allocate nothing here either. Calls on one device share
     the scratch, so calls that overlap on the GPU must not be issued."""
     _check_qkv(q, k, v)
+    _same_device(q.device, out, lse)
     B, H, L, d = q.shape
-    o = torch.empty_like(q) if out is None else out
-    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    rc = load_library().rsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H, L, d,
-                                            N, int(bool(causal)), _dtype_code(q.dtype),
-                                            ctypes.c_void_p(s.cuda_stream))
+    with torch.cuda.device(q.device):
+        o = torch.empty_like(q) if out is None else out
+        ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        rc = load_library().rsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ls), B, H,
+                                                L, d, N, int(bool(causal)), _dtype_code(q.dtype),
+                                                ctypes.c_void_p(s.cuda_stream))
     if rc != RSA_OK:
         raise RSAError(rc, "rsa_forward_noalloc")
     return o, ls

@@ -123,7 +123,7 @@ def test_plans_fit_their_budget_and_grow_with_it(lib, dtype, bwd):
             assert info["heads_per_group"] == B * H
         assert rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, stats - 1)["fits"] is False
         return
-    sizes = []
+    sizes, groups = [], []
     for budget in [1, 1 << 18, 1 << 20, 1 << 22, 1 << 24, 1 << 26, 1 << 30]:
         n = rsa.workspace_size(B, H, L, d, N, False, dtype, bwd, budget)
         info = rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, n)
@@ -135,13 +135,30 @@ def test_plans_fit_their_budget_and_grow_with_it(lib, dtype, bwd):
         assert Lp % 64 == 0 and Lp >= L
         rows = info["rows_per_group"]
         assert rows == L or rows % 128 == 0
-        # every (head, row) is covered exactly once by the groups
-        if rows == L:
-            assert info["groups"] == -(-B * H // info["heads_per_group"])
-        else:
-            assert info["groups"] == B * H * -(-L // rows)
+        # every (head, row) is covered exactly once by the groups: rectangles of
+        # heads_per_group heads x rows_per_group rows
+        assert info["groups"] == -(-B * H // info["heads_per_group"]) * -(-L // rows)
+        groups.append(info["groups"])
     assert sizes == sorted(sizes)
+    assert groups == sorted(groups, reverse=True)  # a larger budget never needs more groups
     assert rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, sizes[0] - 1)["fits"] is False
+
+
+def test_forward_groups_are_balanced(lib):
+    """The bf16 forward's slab groups are equal rectangles of heads x 128-row tiles, not a set of
+    full groups plus a small tail: for the long-sequence shape (a head's slab is 1.09 GB, over
+    the 1 GiB default) every group holds at least 96 of the 2048 (head, row tile) units."""
+    B, H, L, d, N = 1, 16, 16384, 128, 16
+    n = rsa.workspace_size(B, H, L, d, N, False, torch.bfloat16, False, 0)
+    info = rsa.plan_describe(B, H, L, d, N, False, torch.bfloat16, False, n)
+    assert info["fits"] and n <= (1 << 30)
+    hg, rows = info["heads_per_group"], info["rows_per_group"]
+    tiles = -(-L // 128)
+    rt = rows // 128
+    for g in range(info["groups"]):
+        heads = min(hg, B * H - (g // -(-L // rows)) * hg)
+        t = min(rt, tiles - (g % -(-L // rows)) * rt)
+        assert heads * t >= 96, (g, heads, t)
 
 
 def test_default_plan_is_capped_at_one_gib(lib):
@@ -149,3 +166,33 @@ def test_default_plan_is_capped_at_one_gib(lib):
     assert n <= (1 << 30)
     info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, True, n)
     assert info["fits"]
+
+
+def _fwdn(lib, B=1, H=1, L=128, d=64, N=1, dt=rsa.RSA_BF16, ptr=FAKE, lse=FAKE):
+    return lib.rsa_forward_noalloc(ptr, ptr, ptr, ptr, lse, B, H, L, d, N, 0, dt, None)
+
+
+@pytest.mark.parametrize("bad", [dict(L=100, N=3), dict(B=0), dict(N=0), dict(d=96),
+                                 dict(d=128, dt=rsa.RSA_F32), dict(dt=7), dict(ptr=0),
+                                 dict(lse=0), dict(ptr=FAKE + 8), dict(L=(1 << 22) + 1024),
+                                 dict(B=1 << 12, H=1 << 12, L=1 << 16)])
+def test_noalloc_reports_the_codes_forward_reports(lib, bad):
+    """The allocation-free forward checks its arguments like rsa_forward, in the same order, so
+    the same bad arguments give the same code (and nothing touches a device)."""
+    assert _fwdn(lib, **bad) == _fwd(lib, **bad) != rsa.RSA_OK
+
+
+def test_noalloc_refuses_rows_beyond_its_scratch_before_any_device_call(lib):
+    # rows of 70,000 keys: even one 128-row tile of scores exceeds the 32 MiB scratch
+    assert _fwdn(lib, L=70000, N=1) == rsa.RSA_ERR_WORKSPACE
+
+
+def test_status_hook_rejects_codes_a_kernel_never_reports(lib):
+    assert lib.rsa_debug_report_status(rsa.RSA_ERR_CUDA, None) == rsa.RSA_ERR_INVALID_ARG
+    assert lib.rsa_debug_report_status(-1, None) == rsa.RSA_ERR_INVALID_ARG
+
+
+def test_bindings_refuse_outputs_on_another_device():
+    cpu = torch.empty(4)
+    with pytest.raises(ValueError, match="expected cuda:0"):
+        rsa._same_device(torch.device("cuda", 0), None, cpu)

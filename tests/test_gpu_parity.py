@@ -82,7 +82,7 @@ def check_full(orc, x, got, causal, bwd=True, magnitude_scaled=False):
             check(got[name], ref, x.dtype, name, magnitude_scaled)
 
 
-def check_sampled(orc, x, got, causal, heads, rows, keys):
+def check_sampled(orc, x, got, causal, heads, rows, keys, keys_heads=1):
     for (b, h) in heads:
         o, lse = orc.forward_rows(x.q, x.k, x.v, b, h, rows, causal)
         check(got["O"][b, h, rows], o, x.dtype, f"O[{b},{h}] rows")
@@ -90,10 +90,10 @@ def check_sampled(orc, x, got, causal, heads, rows, keys):
         dq = orc.backward_rows(x.q, x.k, x.v, x.do, b, h, rows, causal)
         check(got["dQ"][b, h, rows], dq, x.dtype, f"dQ[{b},{h}] rows")
     if keys is not None:
-        b, h = heads[0]
-        dk, dv = orc.backward_keys(x.q, x.k, x.v, x.do, b, h, keys, causal)
-        check(got["dK"][b, h, keys], dk, x.dtype, f"dK[{b},{h}] keys")
-        check(got["dV"][b, h, keys], dv, x.dtype, f"dV[{b},{h}] keys")
+        for (b, h) in heads[:keys_heads]:
+            dk, dv = orc.backward_keys(x.q, x.k, x.v, x.do, b, h, keys, causal)
+            check(got["dK"][b, h, keys], dk, x.dtype, f"dK[{b},{h}] keys")
+            check(got["dV"][b, h, keys], dv, x.dtype, f"dV[{b},{h}] keys")
 
 
 def sample(L, seed, n=60, edges=(0, 1)):
@@ -160,24 +160,27 @@ def test_config3_gpt_causal(orc):
 
 def test_config4_long_sequence(orc):
     """B=1 H=16 L=16384 d=128 N=16 bf16, forward slab groups in sequence (1 GiB default
-    workspace): sampled rows of two heads and sampled keys of one head."""
+    workspace): sampled rows and sampled keys of two heads."""
     x = make_inputs(1, 16, 16384, 128, seed=4, dtype="bf16")
     info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, False,
                              rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, False))
     assert info["groups"] > 1  # the forward's slab is processed group by group
     got = run(x, 16, False)
     rows = sample(16384, 4, edges=(0, 1, 1023, 1024))
-    check_sampled(orc, x, got, False, [(0, 0), (0, 13)], rows, keys=sample(16384, 40, n=24))
+    # 60 random keys plus the edges of the sequence and of a chunk, on both sampled heads
+    keys = sample(16384, 40, n=60, edges=(0, 1, 1023, 1024, 8191, 8192))
+    check_sampled(orc, x, got, False, [(0, 0), (0, 13)], rows, keys=keys, keys_heads=2)
     check_invariants(x, got)
 
 
-SWEEP_L = [1024, 2048, 4096, 8192]
+SWEEP_L = [1024, 2048, 4096, 8192, 16384]
 
 
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("L", SWEEP_L)
 def test_sweep_against_oracle_and_n_invariance(orc, L, causal):
-    """B=1 H=16 d=64 bf16: every N in {1,2,4,8,16} agrees with N=1; the oracle checks one head."""
+    """B=1 H=16 d=64 bf16: every N in {1,2,4,8,16} agrees with N=1 on every head; the oracle
+    checks sampled rows and keys of one head at N=16."""
     idx = SWEEP_L.index(L) * 10 + int(causal)
     x = make_inputs(1, 16, L, 64, seed=5 + idx, dtype="bf16")
     base = run(x, 1, causal)
@@ -191,11 +194,32 @@ def test_sweep_against_oracle_and_n_invariance(orc, L, causal):
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_sweep_maximum_length(orc, causal):
-    """The sweep's largest point, L = 32768, N = 16: sampled rows against the oracle."""
+    """The sweep's largest point, L = 32768: every N in {2,4,8,16} agrees with N=1 on every
+    head, and at N = 16 sampled rows of one head agree with the oracle."""
     x = make_inputs(1, 16, 32768, 64, seed=60 + int(causal), dtype="bf16")
+    base = run(x, 1, causal)
+    for N in (2, 4, 8):
+        got = run(x, N, causal)
+        for n in ("O", "dQ", "dK", "dV"):
+            check(got[n], base[n], "bf16", f"{n} N={N} vs N=1")
     got = run(x, 16, causal)
+    for n in ("O", "dQ", "dK", "dV"):
+        check(got[n], base[n], "bf16", f"{n} N=16 vs N=1")
     check_sampled(orc, x, got, causal, [(0, 3)], sample(32768, 7, edges=(0, 77, 16384)), keys=None)
     check_invariants(x, got)
+
+
+def test_device_status_word_is_reported_and_cleared():
+    """The path a kernel takes when a bounded wait gives up: it posts RSA_ERR_TIMEOUT into the
+    device status word, rsa_last_device_status returns it once and clears it. The post here
+    comes from the library's injection hook (a one-thread kernel), so no wait runs out."""
+    assert rsa.last_device_status() == rsa.RSA_OK
+    rsa.debug_report_status(rsa.RSA_ERR_TIMEOUT)
+    assert rsa.last_device_status() == rsa.RSA_ERR_TIMEOUT
+    assert rsa.last_device_status() == rsa.RSA_OK
+    # a later healthy call is unaffected
+    x = make_inputs(1, 1, 256, 64, seed=11, dtype="bf16")
+    run(x, 2, False)
 
 
 # ------------------------------------------------------------------ edge cases

@@ -53,6 +53,7 @@ def _close(got, ref, dtype):
 @pytest.mark.parametrize("dtype,shape,N,causal", [
     ("bf16", (2, 8, 1024, 64), 4, True),    # several slab groups fit in the scratch
     ("bf16", (1, 2, 700, 128), 7, False),
+    ("bf16", (1, 1, 8192, 64), 8, True),    # one head's slab exceeds the scratch: row ranges
     ("f32", (1, 2, 256, 32), 4, False),
 ])
 def test_noalloc_forward_matches_forward_on_two_calls(lib, dtype, shape, N, causal):
@@ -64,6 +65,9 @@ def test_noalloc_forward_matches_forward_on_two_calls(lib, dtype, shape, N, caus
     o_ref, lse_ref = rsa.forward(q, k, v, N, causal)  # caller-allocated workspace
     need = lib.rsa_workspace_size(B, H, L, d, N, int(causal), rsa._dtype_code(tdt), 0, SCRATCH)
     assert 0 < need <= SCRATCH
+    plan = rsa.plan_describe(B, H, L, d, N, causal, tdt, False, SCRATCH)
+    if L == 8192:
+        assert plan["rows_per_group"] < L  # the row-range plan is the one exercised
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
         o = torch.full_like(q, float("nan"))
