@@ -88,7 +88,7 @@ struct BkTile {
 __device__ __forceinline__ bool bk_decode(const SlabArgs &a, int t, BkTile &tl) {
     const int kt = t / a.nh;
     tl.h = t - kt * a.nh;
-    tl.j0 = kt * 128;
+    tl.j0 = a.kcol0 + kt * 128;
     const int nqb = (a.R + 63) / 64;
     int lo = 0;
     if (a.causal) lo = max(0, (tl.j0 - a.r0) / 64);
@@ -256,11 +256,11 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     mbar_arrive_expect_tx(bar, 2 * C::QT_BYTES + 512);
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb) {
-                        tma_load_3d(st + kb * 8192, &mQ, bar, kb * 64, row, bh);
-                        tma_load_3d(st + C::QT_BYTES + kb * 8192, &mdO, bar, kb * 64, row, bh);
+                        tma_load_3d(st + kb * 8192, &mQ, bar, kb * 64, row - a.qrow0, bh);
+                        tma_load_3d(st + C::QT_BYTES + kb * 8192, &mdO, bar, kb * 64, row - a.qrow0, bh);
                     }
-                    tma_load_3d(st + C::STAT_OFF, &mStat, bar, row, bh, 0);        // lse * log2(e)
-                    tma_load_3d(st + C::STAT_OFF + 256, &mStat, bar, row, bh, 1);  // D
+                    tma_load_3d(st + C::STAT_OFF, &mStat, bar, row - a.qrow0, bh, 0);        // lse * log2(e)
+                    tma_load_3d(st + C::STAT_OFF + 256, &mStat, bar, row - a.qrow0, bh, 1);  // D
                     issued[p.stage] = true;
                     ipar[p.stage] = p.phase;
                     pipe_next(p, C::STAGES);
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tmem_ld32(t_s, rs);
                 tmem_ld32(t_s + 64, rd);
                 tmem_ld_wait();
-                const bool masked = (a.causal && ic < tl.j0 + 128) || tl.j0 + 128 > a.L ||
+                const bool masked = (a.causal && ic < tl.j0 + 128) || tl.j0 + 128 > a.kend ||
                                     ic + 32 > r_end;
                 // row statistics of this warp's 32 queries, loaded with the step's Q/dO stage
                 const float *stat = reinterpret_cast<const float *>(
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 if (!masked)
                     epi_compute<false>(rs, rd, stat, sl2, 0, 0, 0, 0, 0, wp, wd);
                 else
-                    epi_compute<true>(rs, rd, stat, sl2, j, ic, a.L, r_end, a.causal, wp, wd);
+                    epi_compute<true>(rs, rd, stat, sl2, j, ic, a.kend, r_end, a.causal, wp, wd);
                 // P^T and dS^T over the columns just read, as the dV/dK MMAs' A operands
                 tmem_st16(t_s, wp);
                 tmem_st16(t_s + 64, wd);
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     uint32_t r[32];
                     tmem_ld32(tmem + lane_base + 256 + which * D + col, r);
                     tmem_ld_wait();
-                    if (jw >= a.L) continue;  // the whole 32-row box lies past the sequence
+                    if (jw >= a.kend) continue;  // the whole 32-row box lies past the key window
                     uint8_t *buf = obase + obuf * 2048;
                     obuf = obuf + 1 == C::OUT_BUFS ? 0 : obuf + 1;
                     if (lane == 0) bulk_wait_read<C::OUT_BUFS - 1>();
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                     fence_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_3d(which ? &mdK : &mdV, buf, col, jw, bh);
+                        tma_store_3d(which ? &mdK : &mdV, buf, col, jw - a.kcol0, bh);
                         bulk_commit();
                     }
                 }
@@ -660,9 +660,9 @@ struct BrTile {
 __device__ __forceinline__ void br_decode(const SlabArgs &a, int t, int kn, BrTile &tl) {
     const int u = t / a.nh;
     tl.h = t - u * a.nh;
-    const int nqt = (a.L + 127) / 128;
+    const int nqt = (a.R + 127) / 128;
     const int qt = a.causal ? nqt - 1 - u : u;
-    tl.i0 = qt * 128;
+    tl.i0 = a.r0 + qt * 128;
     const int end = a.causal ? min(a.L, tl.i0 + 128) : a.L;
     tl.cnt = (end + kn - 1) / kn;
     const int n = tl.i0 / a.c;
@@ -780,9 +780,11 @@ __global__ void __launch_bounds__(kBrThreads, 1)
                     mbar_arrive_expect_tx(bar, C::SLOT_BYTES);
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb) {
-                        tma_load_3d(slot + kb * 16384, &mQ, bar, kb * 64, tl.i0, bh);
-                        tma_load_3d(slot + C::QT_BYTES + kb * 16384, &mdO, bar, kb * 64, tl.i0, bh);
-                        tma_load_3d(slot + 2 * C::QT_BYTES + kb * 16384, &mO, bar, kb * 64, tl.i0, bh);
+                        tma_load_3d(slot + kb * 16384, &mQ, bar, kb * 64, tl.i0 - a.qrow0, bh);
+                        tma_load_3d(slot + C::QT_BYTES + kb * 16384, &mdO, bar, kb * 64,
+                                    tl.i0 - a.qrow0, bh);
+                        tma_load_3d(slot + 2 * C::QT_BYTES + kb * 16384, &mO, bar, kb * 64,
+                                    tl.i0 - a.qrow0, bh);
                     }
                     qissued[qs.stage] = true;
                     qpar[qs.stage] = qs.phase;
@@ -930,7 +932,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             const int rt = 32 * q + lane;    // this thread's row of the tile
             const int iw = tl.i0 + 32 * q;  // this warp's first query row
             const int i = iw + lane;         // this thread's query row
-            const float lse_i = i < a.L ? lse[static_cast<size_t>(bh) * a.L + i] : 0.f;
+            const float lse_i =
+                i < a.r0 + a.R ? lse[static_cast<size_t>(bh) * a.Lq + (i - a.qrow0)] : 0.f;
             if (!warp_wait(&ctl->qfull[qs.stage], qs.phase, &ctl->abort)) break;
             // D_i = dO_i . O_i: this warp's half of the columns, then the other half's partial
             // through shared memory (rows past L are zero-filled, so their D is 0)
@@ -961,9 +964,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             if (lane == 0) mbar_arrive(&ctl->qempty[qs.stage]);
             pipe_next(qs, C::Q_SLOTS);
             // the rows' statistics for the key-major kernel, padded with zeros to Lp
-            if (hf == 0 && i < a.Lp) {
-                lse2_out[static_cast<size_t>(bh) * a.Lp + i] = lse2;
-                d_out[static_cast<size_t>(bh) * a.Lp + i] = Di;
+            if (hf == 0 && i - a.qrow0 < a.Lpq) {
+                lse2_out[static_cast<size_t>(bh) * a.Lpq + (i - a.qrow0)] = lse2;
+                d_out[static_cast<size_t>(bh) * a.Lpq + (i - a.qrow0)] = Di;
             }
             for (int s = 0; s < tl.cnt; ++s) {
                 const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
@@ -1016,7 +1019,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->accempty);
-            if (iw >= a.L) continue;  // the whole 32-row box lies past the sequence
+            if (iw >= a.r0 + a.R) continue;  // the whole 32-row box lies past the rows held
 #pragma unroll
             for (int cc = 0; cc < D / 64; ++cc) {
                 uint8_t *buf = obase + obuf * 2048;
@@ -1036,7 +1039,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mdQ, buf, hf * (D / 2) + 32 * cc, iw, bh);
+                    tma_store_3d(&mdQ, buf, hf * (D / 2) + 32 * cc, iw - a.qrow0, bh);
                     bulk_commit();
                 }
             }

@@ -47,8 +47,9 @@ struct QkTile {
     int h, i0, ct;
 };
 
-// Tiles are (head, 128-row tile, 256-column tile); causal tiles right of the diagonal are
-// skipped. The column tiles of a row tile start at the block holding its own chunk's keys.
+// Tiles are (head, 128-row tile, 256-column tile of the key window [kcol0, kend)); causal
+// tiles right of the diagonal are skipped. The column tiles of a row tile start at the block
+// holding its own chunk's keys.
 __device__ __forceinline__ bool qk_decode(const SlabArgs &a, int t, QkTile &tl) {
     const int per_head = a.nRT * a.nCT;
     tl.h = t / per_head;
@@ -57,10 +58,10 @@ __device__ __forceinline__ bool qk_decode(const SlabArgs &a, int t, QkTile &tl) 
     const int cti = rem - rt * a.nCT;
     tl.i0 = a.r0 + rt * 128;
     int live = a.nCT;
-    if (a.causal) live = min(a.nCT, (min(a.L, tl.i0 + 128) + 255) / 256);
+    if (a.causal) live = min(a.nCT, (min(a.kend, tl.i0 + 128) - a.kcol0 + 255) / 256);
     if (cti >= live) return false;
     const int n = tl.i0 / a.c;
-    const int first = min((n * a.c) / 256, live - 1);
+    const int first = min(max((n * a.c - a.kcol0) / 256, 0), live - 1);
     tl.ct = ring_block(first, cti, live);
     return true;
 }
@@ -122,8 +123,9 @@ __global__ void __launch_bounds__(kQkThreads, 1)
                     uint8_t *sa = stages + p.stage * C::STAGE_BYTES;
                     uint64_t *bar = &ctl->full[p.stage];
                     mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                    tma_load_3d(sa, &mQ, bar, kb * 64, tl.i0, a.bh0 + tl.h);
-                    tma_load_3d(sa + C::A_BYTES, &mK, bar, kb * 64, tl.ct * C::BN, a.bh0 + tl.h);
+                    tma_load_3d(sa, &mQ, bar, kb * 64, tl.i0 - a.qrow0, a.bh0 + tl.h);
+                    tma_load_3d(sa + C::A_BYTES, &mK, bar, kb * 64, a.kcol0 + tl.ct * C::BN,
+                                a.bh0 + tl.h);
                     issued[p.stage] = true;
                     ipar[p.stage] = p.phase;
                     pipe_next(p, C::STAGES);
@@ -190,10 +192,10 @@ __global__ void __launch_bounds__(kQkThreads, 1)
                 uint32_t r[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * C::BN + col, r);
                 tmem_ld_wait();
-                const int j0 = tl.ct * C::BN + col;
+                const int j0 = a.kcol0 + tl.ct * C::BN + col;
                 float v[32];
                 float cm = -INFINITY;
-                if (j0 + 32 <= a.L && (!a.causal || j0 + 31 <= i_min)) {
+                if (j0 + 32 <= a.kend && (!a.causal || j0 + 31 <= i_min)) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         v[e] = __uint_as_float(r[e]) * sl2;
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kQkThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int j = j0 + e;
-                        const bool live = j < a.L && !(a.causal && j > i);
+                        const bool live = j < a.kend && !(a.causal && j > i);
                         v[e] = live ? __uint_as_float(r[e]) * sl2 : -INFINITY;
                         cm = fmaxf(cm, v[e]);
                     }
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(kQkThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mS, buf, j0, tl.i0 - a.r0 + 32 * q, tl.h);
+                    tma_store_3d(&mS, buf, j0 - a.kcol0, tl.i0 - a.r0 + 32 * q, tl.h);
                     bulk_commit();
                 }
             }
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kQkThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
             if (i < a.r0 + a.R)
-                a.stats[(static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat + 2 * tl.ct + hf] =
+                a.stats[(static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat + a.stat0 + 2 * tl.ct + hf] =
                     make_float2(run_m, run_l);
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
@@ -451,8 +453,14 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
             // the row's softmax statistics from the slab GEMM's partials
             float m = 0.f, inv = 0.f;
             if (i < a.r0 + a.R) {
-                const int nlive =
-                    a.causal ? 2 * ((min(a.L, (i / 128) * 128 + 128) + 255) / 256) : a.nStat;
+                // causal: the partials of the windows up to the one holding the tile's last
+                // live key (each window holds 2 * ceil(wlen / 256) slots)
+                int nlive = a.nStat;
+                if (a.causal) {
+                    const int end = min(a.L, (i / 128) * 128 + 128);
+                    const int wl = (end - 1) / a.wlen;
+                    nlive = wl * 2 * ((a.wlen + 255) / 256) + 2 * ((end - wl * a.wlen + 255) / 256);
+                }
                 const float2 *st = a.stats + (static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat;
                 float l = 0.f;
                 m = -INFINITY;
@@ -461,7 +469,9 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                     softmax_combine(m, l, x.x, x.y);
                 }
                 inv = 1.f / l;
-                if (hf == 0) lse[static_cast<size_t>(bh) * a.L + i] = (m + __log2f(l)) * 0.6931471805599453f;
+                if (hf == 0)
+                    lse[static_cast<size_t>(bh) * a.Lq + (i - a.qrow0)] =
+                        (m + __log2f(l)) * 0.6931471805599453f;
             }
             for (int s = 0; s < tl.nkb; ++s) {
                 const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
@@ -520,7 +530,7 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mO, buf, hf * (D / 2) + 32 * cc, iw, bh);
+                    tma_store_3d(&mO, buf, hf * (D / 2) + 32 * cc, iw - a.qrow0, bh);
                     bulk_commit();
                 }
             }

@@ -8,6 +8,7 @@
 // group so that the workspace stays within a budget. A group is a set of whole heads, or a
 // range of rows (a multiple of 128) of one head when a whole head does not fit.
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 
 #include <math.h>
 #include <mutex>
@@ -16,6 +17,7 @@
 #include <vector>
 
 #include "../../include/rsa.h"
+#include "../../include/rsa_sp.h"
 #include "rsa_internal.h"
 
 namespace rsa {
@@ -282,12 +284,12 @@ rsa_status_t device_state(DeviceState **out) {
 
 enum Kind {
     K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_BWD_ROWS,
-    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_FWD_STATS, K_FWD_PV, K_COUNT
+    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_FWD_STATS, K_FWD_PV, K_SP_ACC, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
     "qk_slab", "slab_softmax", "pv_softmax", "rowdot", "bwd_keys", "bwd_rows",
     "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows",
-    "fwd_stats", "fwd_pv"};
+    "fwd_stats", "fwd_pv", "sp_accumulate"};
 
 struct ProfRec {
     int kind;
@@ -389,6 +391,8 @@ SlabArgs slab_args(const Plan &p, const Group &G, int *status) {
     a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(p.d)));
     a.nRT = (G.R + 127) / 128;
     a.status = status;
+    a.qrow0 = 0, a.Lq = p.L, a.Lpq = p.Lp;
+    a.kcol0 = 0, a.kend = p.L, a.wlen = p.L, a.stat0 = 0;
     return a;
 }
 
@@ -402,6 +406,119 @@ rsa_status_t check_common(const Plan &p, void *ws, size_t ws_bytes) {
     if (p.total > ws_bytes) return RSA_ERR_WORKSPACE;
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return RSA_ERR_INVALID_ARG;
     return RSA_OK;
+}
+
+
+// ---------------------------------------------------------------- sequence-parallel layout
+
+// One rank's share of the sequence-parallel ring: rows [rank c, (rank + 1) c) of every head.
+struct SpLayout {
+    long long BH;
+    int c, Lp, nCT, nStat;
+    size_t slab_bytes, part_bytes, fwd_total, bwd_total;
+};
+
+bool sp_args_ok(int B, int H, int L, int d, int P, int rank, int m, rsa_status_t *why) {
+    if (!args_ok(B, H, L, d, P, RSA_BF16, why)) return false;
+    if (rank < 0 || rank >= P || m < 0 || m >= P) {
+        *why = RSA_ERR_INVALID_ARG;
+        return false;
+    }
+    // whole 128-row tiles per rank; key chunks aligned with the kernels' 64/128-key blocks
+    if ((L / P) % 128 != 0) {
+        *why = RSA_ERR_UNSUPPORTED;
+        return false;
+    }
+    return true;
+}
+
+SpLayout sp_layout(int B, int H, int L, int P) {
+    SpLayout y{};
+    y.BH = static_cast<long long>(B) * H;
+    y.c = L / P;
+    y.Lp = L;  // a multiple of 128
+    y.nCT = (y.c + 255) / 256;
+    y.nStat = P * 2 * y.nCT;
+    y.slab_bytes = align_up(size_t(y.BH) * y.c * y.Lp * 4, kAlign);
+    y.part_bytes = align_up(size_t(y.BH) * y.c * y.nStat * 8, kAlign);
+    y.fwd_total = y.slab_bytes + y.part_bytes;
+    y.bwd_total = align_up(size_t(2) * y.BH * y.c * 4, kAlign);
+    return y;
+}
+
+SlabArgs sp_slab_args(const SpLayout &y, int L, int d, int P, int rank, int causal, int *status) {
+    SlabArgs a{};
+    a.L = L, a.Lp = y.Lp, a.N = P, a.c = y.c, a.causal = causal ? 1 : 0, a.d = d;
+    a.bh0 = 0, a.nh = static_cast<int>(y.BH), a.r0 = rank * y.c, a.R = y.c;
+    a.scale = static_cast<float>(1.0 / sqrt(static_cast<double>(d)));
+    a.nRT = y.c / 128;
+    a.status = status;
+    a.qrow0 = rank * y.c, a.Lq = y.c, a.Lpq = y.c;
+    a.kcol0 = 0, a.kend = L, a.wlen = y.c, a.stat0 = 0;
+    a.nCT = y.nCT, a.nStat = y.nStat;
+    return a;
+}
+
+// bf16 [BH][rows][d] tensor, boxes of 64 columns x box_rows rows (128-byte swizzle)
+bool map_rows(CUtensorMap *m, const void *base, long long BH, int rows, int d, uint32_t box_rows) {
+    return map3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d, rows, BH, uint64_t(d) * 2,
+                 uint64_t(rows) * d * 2, 64, box_rows);
+}
+
+// bf16 [BH][rows][d] output written by 32 x 32 TMA stores (64-byte swizzle)
+bool map_rows_out(CUtensorMap *m, void *base, long long BH, int rows, int d) {
+    return map3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d, rows, BH, uint64_t(d) * 2,
+                 uint64_t(rows) * d * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+bool ws_ok(const void *ws) { return ws && (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) == 0; }
+
+// The travelling accumulator of the backward ring (rsa_sp_accumulate): 8 elements per thread
+// where the tail allows, one otherwise.
+__global__ void sp_accumulate_kernel(float *__restrict__ acc, const __nv_bfloat16 *__restrict__ part,
+                                     __nv_bfloat16 *__restrict__ out, long long n, int first) {
+    const long long nv = n / 8;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nv; v += stride) {
+        float x[8];
+        if (first) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        } else {
+            const float4 a0 = reinterpret_cast<const float4 *>(acc)[2 * v];
+            const float4 a1 = reinterpret_cast<const float4 *>(acc)[2 * v + 1];
+            x[0] = a0.x, x[1] = a0.y, x[2] = a0.z, x[3] = a0.w;
+            x[4] = a1.x, x[5] = a1.y, x[6] = a1.z, x[7] = a1.w;
+        }
+        if (part) {
+            const uint4 p = reinterpret_cast<const uint4 *>(part)[v];
+            const __nv_bfloat162 *pb = reinterpret_cast<const __nv_bfloat162 *>(&p);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(pb[e]);
+                x[2 * e] += f.x;
+                x[2 * e + 1] += f.y;
+            }
+        }
+        reinterpret_cast<float4 *>(acc)[2 * v] = make_float4(x[0], x[1], x[2], x[3]);
+        reinterpret_cast<float4 *>(acc)[2 * v + 1] = make_float4(x[4], x[5], x[6], x[7]);
+        if (out) {
+            uint4 o;
+            uint32_t *ow = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+                ow[e] = *reinterpret_cast<uint32_t *>(&b);
+            }
+            reinterpret_cast<uint4 *>(out)[v] = o;
+        }
+    }
+    for (long long i = nv * 8 + blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n; i += stride) {
+        float x = first ? 0.f : acc[i];
+        if (part) x += __bfloat162float(part[i]);
+        acc[i] = x;
+        if (out) out[i] = __float2bfloat16_rn(x);
+    }
 }
 
 }  // namespace
@@ -676,6 +793,160 @@ rsa_status_t rsa_backward(const void *Q, const void *K, const void *V, const voi
     // key-major ring: P^T, dP^T -> dS^T in TMEM; dV_m, dK_m over all query blocks
     RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK128, mV128, mQ64, mdO64, mStat64, mdK, mdV, a,
                                                 dev->sms, s));
+    return RSA_OK;
+}
+
+// ---------------------------------------------------------------- sequence-parallel steps
+
+size_t rsa_sp_workspace_size(int B, int H, int L, int d, int P, int causal, int for_backward) {
+    (void)causal;
+    rsa_status_t why;
+    if (!sp_args_ok(B, H, L, d, P, 0, 0, &why)) return 0;
+    const SpLayout y = sp_layout(B, H, L, P);
+    return for_backward ? y.bwd_total : y.fwd_total;
+}
+
+rsa_status_t rsa_sp_scores(const void *Q, const void *Kfull, int B, int H, int L, int d, int P,
+                           int rank, int m, int causal, void *workspace, size_t ws_bytes,
+                           void *stream) {
+    rsa_status_t why;
+    if (!sp_args_ok(B, H, L, d, P, rank, m, &why)) return why;
+    if (!Q || !Kfull || !aligned16(Q) || !aligned16(Kfull) || !ws_ok(workspace))
+        return RSA_ERR_INVALID_ARG;
+    const SpLayout y = sp_layout(B, H, L, P);
+    if (ws_bytes < y.fwd_total) return RSA_ERR_WORKSPACE;
+    if (causal && m > rank) return RSA_OK;  // the whole window lies right of the diagonal
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    SlabArgs a = sp_slab_args(y, L, d, P, rank, causal, dev->status);
+    a.kcol0 = m * y.c, a.kend = (m + 1) * y.c, a.stat0 = m * 2 * y.nCT;
+    a.stats = reinterpret_cast<float2 *>(ws + y.slab_bytes);
+    a.ntiles = a.nh * a.nRT * a.nCT;
+    // the slab window of chunk m: columns [m c, (m + 1) c) of the rank's [BH][c][L] scores; the
+    // map's extent clips the stores of a tile that reaches past the window
+    const uint64_t pitch = uint64_t(y.Lp) * 4;
+    CUtensorMap mQ, mK, mS;
+    if (!map_rows(&mQ, Q, y.BH, y.c, d, 128) || !map_rows(&mK, Kfull, y.BH, L, d, 256) ||
+        !map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws + size_t(m) * y.c * 4, y.c, y.c, y.BH,
+               pitch, pitch * y.c, 32, 32))
+        return RSA_ERR_CUDA;
+    RSA_LAUNCH(K_QK_SLAB, rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
+    return RSA_OK;
+}
+
+rsa_status_t rsa_sp_softmax_pv(const void *Vfull, void *O, float *lse, int B, int H, int L, int d,
+                               int P, int rank, int causal, void *workspace, size_t ws_bytes,
+                               void *stream) {
+    rsa_status_t why;
+    if (!sp_args_ok(B, H, L, d, P, rank, 0, &why)) return why;
+    if (!Vfull || !O || !lse || !aligned16(Vfull) || !aligned16(O) || !aligned16(lse) ||
+        !ws_ok(workspace))
+        return RSA_ERR_INVALID_ARG;
+    const SpLayout y = sp_layout(B, H, L, P);
+    if (ws_bytes < y.fwd_total) return RSA_ERR_WORKSPACE;
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    SlabArgs a = sp_slab_args(y, L, d, P, rank, causal, dev->status);
+    a.stats = reinterpret_cast<float2 *>(ws + y.slab_bytes);
+    a.ntiles = a.nh * a.nRT;
+    const uint64_t pitch = uint64_t(y.Lp) * 4;
+    CUtensorMap mS, mV, mO;
+    if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws, y.Lp, y.c, y.BH, pitch, pitch * y.c, 32,
+               128) ||
+        !map_rows(&mV, Vfull, y.BH, L, d, 64) || !map_rows_out(&mO, O, y.BH, y.c, d))
+        return RSA_ERR_CUDA;
+    RSA_LAUNCH(K_PV, rsa::launch_pv_softmax(mS, mV, mO, lse, a, dev->sms, s));
+    return RSA_OK;
+}
+
+rsa_status_t rsa_sp_backward_rows(const void *Q, const void *Kfull, const void *Vfull,
+                                  const void *O, const void *dO, const float *lse, void *dQ,
+                                  int B, int H, int L, int d, int P, int rank, int causal,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+    rsa_status_t why;
+    if (!sp_args_ok(B, H, L, d, P, rank, 0, &why)) return why;
+    const void *ptrs[] = {Q, Kfull, Vfull, O, dO, lse, dQ};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return RSA_ERR_INVALID_ARG;
+    if (!ws_ok(workspace)) return RSA_ERR_INVALID_ARG;
+    const SpLayout y = sp_layout(B, H, L, P);
+    if (ws_bytes < y.bwd_total) return RSA_ERR_WORKSPACE;
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *lse2 = static_cast<float *>(workspace);
+    float *Dvec = lse2 + size_t(y.BH) * y.c;
+    SlabArgs a = sp_slab_args(y, L, d, P, rank, causal, dev->status);
+    a.ntiles = a.nh * a.nRT;
+    const uint32_t kn = d == 64 ? 128 : 64;  // keys per step of the query-major kernel
+    CUtensorMap mQ, mdO, mO, mK, mV, mdQ;
+    if (!map_rows(&mQ, Q, y.BH, y.c, d, 128) || !map_rows(&mdO, dO, y.BH, y.c, d, 128) ||
+        !map_rows(&mO, O, y.BH, y.c, d, 128) || !map_rows(&mK, Kfull, y.BH, L, d, kn) ||
+        !map_rows(&mV, Vfull, y.BH, L, d, kn) || !map_rows_out(&mdQ, dQ, y.BH, y.c, d))
+        return RSA_ERR_CUDA;
+    RSA_LAUNCH(K_BWD_ROWS, rsa::launch_bwd_rows(mQ, mdO, mO, mK, mV, mdQ, lse, lse2, Dvec, a,
+                                                dev->sms, s));
+    return RSA_OK;
+}
+
+rsa_status_t rsa_sp_backward_keys(const void *Q, const void *Kfull, const void *Vfull,
+                                  const void *dO, void *dK_part, void *dV_part, int B, int H,
+                                  int L, int d, int P, int rank, int m, int causal,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+    rsa_status_t why;
+    if (!sp_args_ok(B, H, L, d, P, rank, m, &why)) return why;
+    const void *ptrs[] = {Q, Kfull, Vfull, dO, dK_part, dV_part};
+    for (const void *q : ptrs)
+        if (!q || !aligned16(q)) return RSA_ERR_INVALID_ARG;
+    if (!ws_ok(workspace)) return RSA_ERR_INVALID_ARG;
+    const SpLayout y = sp_layout(B, H, L, P);
+    if (ws_bytes < y.bwd_total) return RSA_ERR_WORKSPACE;
+    if (causal && m > rank) return RSA_OK;  // no row of this rank sees a key of chunk m
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *lse2 = static_cast<float *>(workspace);
+    SlabArgs a = sp_slab_args(y, L, d, P, rank, causal, dev->status);
+    a.kcol0 = m * y.c, a.kend = (m + 1) * y.c;
+    a.ntiles = a.nh * (y.c / 128);
+    a.mode = 0;
+    const uint64_t stat_pitch = uint64_t(y.c) * 4;
+    CUtensorMap mK, mV, mQ, mdO, mStat, mdK, mdV;
+    if (!map_rows(&mK, Kfull, y.BH, L, d, 128) || !map_rows(&mV, Vfull, y.BH, L, d, 128) ||
+        !map_rows(&mQ, Q, y.BH, y.c, d, 64) || !map_rows(&mdO, dO, y.BH, y.c, d, 64) ||
+        !map3d(&mStat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lse2, y.c, y.BH, 2, stat_pitch,
+               stat_pitch * y.BH, 64, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !map_rows_out(&mdK, dK_part, y.BH, y.c, d) || !map_rows_out(&mdV, dV_part, y.BH, y.c, d))
+        return RSA_ERR_CUDA;
+    RSA_LAUNCH(K_BWD_KEYS, rsa::launch_bwd_keys(mK, mV, mQ, mdO, mStat, mdK, mdV, a, dev->sms, s));
+    return RSA_OK;
+}
+
+rsa_status_t rsa_sp_accumulate(float *acc, const void *part, void *out, long long n, int first,
+                               void *stream) {
+    if (!acc || n < 0 || !aligned16(acc) || (part && !aligned16(part)) || (out && !aligned16(out)))
+        return RSA_ERR_INVALID_ARG;
+    if (n == 0) return RSA_OK;
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long work = (n + 7) / 8;
+    long long blocks = (work + 255) / 256;
+    const long long cap = static_cast<long long>(dev->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    RSA_LAUNCH(K_SP_ACC, (sp_accumulate_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+                              acc, static_cast<const __nv_bfloat16 *>(part),
+                              static_cast<__nv_bfloat16 *>(out), n, first ? 1 : 0),
+                          cudaGetLastError()));
     return RSA_OK;
 }
 

@@ -60,6 +60,14 @@ struct SlabArgs {
     int nStat;      // forward: per-row softmax partials (one per 128 key columns)
     float2 *stats;  // forward: [nh][R][nStat] (max, sum of 2^(s - max)) in base-2 units
     int *status; // device status word
+    // Views of a sequence-parallel rank (the defaults, in brackets, give the whole problem):
+    int qrow0;   // first query row held: Q, O, dO, dQ and lse are stored at row i - qrow0 [0]
+    int Lq;      // rows per head of that storage [L]
+    int Lpq;     // rows per head of the backward's row statistics (padded to 64) [Lp]
+    int kcol0;   // key window [kcol0, kend) of ring pass 1 and of the key-major backward [0]
+    int kend;    // [L]
+    int wlen;    // keys per window of the softmax partials' layout [L]
+    int stat0;   // first softmax-partial slot of this window [0]
 };
 
 // ---- bf16 tensor-core kernels (kernels_tc.cu) -------------------------------------------
