@@ -22,8 +22,8 @@
 // statistics per step); warp 1 owns TMEM and lane 0 issues tcgen05.mma; warps 2..9 are the
 // epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (keys) and query columns 32*((w-2)/4)..+31.
 // The S^T/dP^T accumulators are double-buffered and the MMA warp issues a step's S^T/dP^T
-// ahead of the previous step's dV/dK (two steps ahead for d = 64, one for d = 128), so the
-// tensor core works on one step while the epilogue works on another. MMAs of one thread
+// two steps ahead of its dV/dK, so the tensor core works on one step while the epilogue works
+// on another. MMAs of one thread
 // execute in issue order, so step t's dV/dK MMAs read P^T/dS^T of buffer b before step t+2's
 // S^T/dP^T MMAs overwrite it.
 #include "tc_common.cuh"
@@ -40,11 +40,16 @@ template <int D>
 struct BkCfg {
     static constexpr int QB = 64;                        // query rows per step
     static constexpr int KV_BYTES = 128 * D * 2;         // resident [128 keys][D] tile
-    static constexpr int KV_SLOTS = 2;
+    // d = 128: one K/V slot (the next unit's K/V load waits for the unit's last S^T/dP^T
+    // MMAs, once per 128-key unit) buys four Q/dO stages: a stage is held from its S^T/dP^T
+    // MMAs to its dV/dK MMAs, about a step and a half, so with two stages the producer could
+    // not load step t + 2 before step t's dV/dK MMAs had finished and the MMA thread waited
+    // for the load (measured: about a third of every step)
+    static constexpr int KV_SLOTS = D == 64 ? 2 : 1;
     static constexpr int QT_BYTES = QB * D * 2;          // [64 queries][D] tile
     static constexpr int STAT_OFF = 2 * QT_BYTES;        // then lse*log2(e) [64] and D [64]
     static constexpr int STAGE_BYTES = 2 * QT_BYTES + 1024;
-    static constexpr int STAGES = D == 64 ? 5 : 2;
+    static constexpr int STAGES = D == 64 ? 5 : 4;
     static constexpr int OUT_BUFS = D == 64 ? 2 : 1;     // 2 KB staging buffers per warp
     static constexpr int OFF_KV = 0;
     static constexpr int OFF_STAGE = OFF_KV + KV_SLOTS * 2 * KV_BYTES;
@@ -274,10 +279,13 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0 && C::KV_TMEM) {
-            // d = 64: S^T/dP^T run two steps ahead of dV/dK. Every barrier poll of this thread
-            // waits for the MMAs it has in flight, so the loop polls once per step: pready(g),
-            // which the epilogue posts only once the Q/dO stage of step g + 2 has landed too.
+        if (lane == 0) {
+            // S^T/dP^T run two steps ahead of dV/dK. Every barrier poll of this thread waits
+            // for the MMAs it has in flight (the pipe then idles until the next issue), so the
+            // loop polls once per step: pready(g), which the epilogue posts only once the Q/dO
+            // stage of step g + 2 has landed too. d = 64: the unit's K and V are copied into
+            // TMEM and the S^T/dP^T MMAs take A from there; d = 128: A comes from the unit's
+            // K/V slot in shared memory, released after the unit's last S^T/dP^T MMAs.
             constexpr uint64_t KM = sdesc_const(16, 1024);
             constexpr uint64_t MN = sdesc_const(8192, 1024);
             const uint32_t id_s = idesc_bf16_f32(128, C::QB, 0, 0);
@@ -306,21 +314,26 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             Cursor gr = is;
             bool has_is = seek(is), has_gr = seek(gr);
             Pipe kv{0, 0};
+            uint32_t kslot = 0;  // d = 128: the K/V slot of the unit under `is`
             uint32_t gi = 0, gg = 0, acc_ph = 0;
             auto issue_s = [&]() -> bool {  // S^T, dP^T of the step under `is`, buffer gi & 1
                 if (is.s == 0) {
-                    // K, V -> TMEM (after every earlier S^T/dP^T MMA, in issue order)
                     if (!mbar_wait(&ctl->kvfull[kv.stage], kv.phase, &ctl->abort)) return false;
                     tc_fence_after();
-                    const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
-                    const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, ks + C::KV_BYTES);
+                    if (C::KV_TMEM) {
+                        // K, V -> TMEM (after every earlier S^T/dP^T MMA, in issue order)
+                        const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
+                        const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, ks + C::KV_BYTES);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        tc_cp_128x256b(tmem + C::T_K + 8 * k, d_k + 2 * k);
-                        tc_cp_128x256b(tmem + C::T_V + 8 * k, d_v + 2 * k);
+                        for (int k = 0; k < D / 16; ++k) {
+                            tc_cp_128x256b(tmem + C::T_K + 8 * k, d_k + 2 * k);
+                            tc_cp_128x256b(tmem + C::T_V + 8 * k, d_v + 2 * k);
+                        }
+                        tc_commit(&ctl->kvempty[kv.stage]);
+                        pipe_next(kv, C::KV_SLOTS);
+                    } else {
+                        kslot = kv.stage;
                     }
-                    tc_commit(&ctl->kvempty[kv.stage]);
-                    pipe_next(kv, C::KV_SLOTS);
                 }
                 // the first two stages are not vouched for by a pready
                 if (gi < 2 && !mbar_wait(&ctl->full[is.p.stage], is.p.phase, &ctl->abort))
@@ -329,12 +342,30 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const uint32_t st = smem_addr(smem + C::OFF_STAGE + is.p.stage * C::STAGE_BYTES);
                 const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
                 const uint32_t t_s = tmem + 128 * (gi & 1u), t_p = t_s + 64;
+                if (C::KV_TMEM) {
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    tc_mma_bf16_ts(t_s, tmem + C::T_K + 8 * k, d_q + 2 * k, id_s, k ? 1u : 0u);
-                    tc_mma_bf16_ts(t_p, tmem + C::T_V + 8 * k, d_do + 2 * k, id_s, k ? 1u : 0u);
+                    for (int k = 0; k < D / 16; ++k) {
+                        tc_mma_bf16_ts(t_s, tmem + C::T_K + 8 * k, d_q + 2 * k, id_s, k ? 1u : 0u);
+                        tc_mma_bf16_ts(t_p, tmem + C::T_V + 8 * k, d_do + 2 * k, id_s, k ? 1u : 0u);
+                    }
+                } else {
+                    const uint32_t ks = smem_addr(smem + C::OFF_KV + kslot * 2 * C::KV_BYTES);
+                    const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, ks + C::KV_BYTES);
+#pragma unroll
+                    for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t en = (kb | k) != 0 ? 1u : 0u;
+                            const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
+                            tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
+                            tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
+                        }
                 }
                 tc_commit(&ctl->sfull[gi & 1u]);
+                if (!C::KV_TMEM && is.s == is.tl.cnt - 1) {
+                    tc_commit(&ctl->kvempty[kv.stage]);  // the unit's last reader of its K/V
+                    pipe_next(kv, C::KV_SLOTS);
+                }
                 ++gi;
                 has_is = advance(is);
                 return true;
@@ -369,88 +400,6 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             }
             tc_commit(&ctl->drain);
             drain_wait(&ctl->drain, 0);
-        } else if (lane == 0) {
-            constexpr uint64_t KM = sdesc_const(16, 1024);    // K-major, 128-byte swizzle
-            constexpr uint64_t MN = sdesc_const(8192, 1024);  // MN-major, 64-wide blocks 8 KB apart
-            const uint32_t id_s = idesc_bf16_f32(128, C::QB, 0, 0);  // S^T, dP^T
-            const uint32_t id_g = idesc_bf16_f32(128, D, 0, 1);      // dV, dK (A in TMEM)
-            const uint32_t t_dv = tmem + 256, t_dk = tmem + 256 + D;
-            Pipe p{0, 0}, kv{0, 0};
-            uint32_t gstep = 0, acc_ph = 0;
-            bool ok = true;
-            // dV/dK work of the previous step, issued after the next step's S^T/dP^T
-            bool pend = false, pend_first = false;
-            int pend_stage = 0;
-            uint32_t pend_b = 0, pend_ph = 0;
-            auto grad = [&](void) -> bool {
-                if (!mbar_wait(&ctl->pready[pend_b], pend_ph, &ctl->abort)) return false;
-                if (pend_first && !mbar_wait(&ctl->accempty, acc_ph ^ 1u, &ctl->abort)) return false;
-                tc_fence_after();
-                const uint32_t st = smem_addr(smem + C::OFF_STAGE + pend_stage * C::STAGE_BYTES);
-                const uint64_t d_do = sdesc(MN, st + C::QT_BYTES), d_q = sdesc(MN, st);
-                const uint32_t t_p = tmem + 128 * pend_b, t_ds = t_p + 64;
-#pragma unroll
-                for (int k = 0; k < C::QB / 16; ++k) {
-                    const uint32_t en = (pend_first && k == 0) ? 0u : 1u;
-                    const uint32_t col = (k >> 1) * 32 + (k & 1) * 8;  // 16 queries per MMA
-                    tc_mma_bf16_ts(t_dv, t_p + col, d_do + 128 * k, id_g, en);
-                    tc_mma_bf16_ts(t_dk, t_ds + col, d_q + 128 * k, id_g, en);
-                }
-                tc_commit(&ctl->empty[pend_stage]);
-                pend = false;
-                return true;
-            };
-            for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
-                BkTile tl;
-                if (!bk_decode(a, t, tl)) continue;
-                if (!mbar_wait(&ctl->kvfull[kv.stage], kv.phase, &ctl->abort)) break;
-                tc_fence_after();
-                const uint32_t ks = smem_addr(smem + C::OFF_KV + kv.stage * 2 * C::KV_BYTES);
-                const uint32_t vs = ks + C::KV_BYTES;
-                const uint64_t d_k = sdesc(KM, ks), d_v = sdesc(KM, vs);
-                for (int s = 0; s < tl.cnt; ++s) {
-                    const uint32_t b = gstep & 1u;
-                    if (!mbar_wait(&ctl->full[p.stage], p.phase, &ctl->abort)) {
-                        ok = false;
-                        break;
-                    }
-                    // buffer b was last read by the dV/dK MMAs of step gstep - 2, issued
-                    // before these (in-order execution)
-                    tc_fence_after();
-                    const uint32_t st = smem_addr(smem + C::OFF_STAGE + p.stage * C::STAGE_BYTES);
-                    const uint32_t t_s = tmem + 128 * b, t_p = t_s + 64;
-                    const uint64_t d_q = sdesc(KM, st), d_do = sdesc(KM, st + C::QT_BYTES);
-#pragma unroll
-                    for (int kb = 0; kb < D / 64; ++kb)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t en = (kb | k) != 0 ? 1u : 0u;
-                            const uint32_t ko = kb * 1024 + 2 * k, qo = kb * 512 + 2 * k;
-                            tc_mma_bf16(t_s, d_k + ko, d_q + qo, id_s, en);
-                            tc_mma_bf16(t_p, d_v + ko, d_do + qo, id_s, en);
-                        }
-                    tc_commit(&ctl->sfull[b]);
-                    if (s == tl.cnt - 1) tc_commit(&ctl->kvempty[kv.stage]);
-                    if (pend && !grad()) {
-                        ok = false;
-                        break;
-                    }
-                    pend = true;
-                    pend_first = s == 0;
-                    pend_stage = p.stage;
-                    pend_b = b;
-                    pend_ph = (gstep >> 1) & 1u;
-                    pipe_next(p, C::STAGES);
-                    ++gstep;
-                }
-                if (!ok) break;
-                if (pend && !grad()) break;
-                tc_commit(&ctl->accfull);
-                acc_ph ^= 1u;
-                pipe_next(kv, C::KV_SLOTS);
-            }
-            tc_commit(&ctl->drain);
-            drain_wait(&ctl->drain, 0);
         }
         __syncwarp();
     } else {
@@ -463,12 +412,11 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         uint32_t gstep = 0, acc_ph = 0;
         Pipe ps{0, 0};  // the Q/dO stage of the current step (same order as the producer's)
         bool ok = true;
-        uint32_t total = 0;  // steps of this CTA (d = 64: pready(g) vouches for stage g + 2)
-        if (C::KV_TMEM)
-            for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-                BkTile tl;
-                if (bk_decode(a, t, tl)) total += tl.cnt;
-            }
+        uint32_t total = 0;  // steps of this CTA (pready(g) vouches for stage g + 2)
+        for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+            BkTile tl;
+            if (bk_decode(a, t, tl)) total += tl.cnt;
+        }
         for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
             BkTile tl;
             if (!bk_decode(a, t, tl)) continue;
@@ -505,7 +453,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tmem_st16(t_s + 64, wd);
                 tmem_st_wait();
                 tc_fence_before();
-                if (C::KV_TMEM && gstep + 2 < total) {
+                if (gstep + 2 < total) {
                     Pipe p2 = ps;
                     pipe_next(p2, C::STAGES);
                     pipe_next(p2, C::STAGES);
@@ -597,7 +545,10 @@ __global__ void __launch_bounds__(kBkThreads, 1)
 // owns TMEM and lane 0 issues tcgen05.mma, warps 2..9 are the epilogue (TMEM lanes
 // 32*(w%4)..+31 are its query rows; it takes keys KN/2*((w-2)/4) .. +KN/2 of each block).
 // S is double-buffered, dP single-buffered: the epilogue loads dP first and releases it
-// (dpfree) before it works on S, so the next block's dP MMAs wait only for that load.
+// (dpfree) before it works on S, so the next block's dP MMAs wait only for that load. (A
+// schedule with dP double-buffered at d = 128, S/dP two steps ahead and one poll per step was
+// measured slower: with three K/V stages the epilogue's wait for the stage two steps ahead put
+// a load latency on every step.)
 // Each poll of a barrier by the MMA thread stalls the tensor pipe for about a hundred cycles,
 // so blocks are as wide as TMEM allows (KN = 128 keys for d = 64). Q and dO are copied into
 // TMEM once per unit (tcgen05.cp) and the S and dP MMAs take them from there: with both

@@ -254,37 +254,39 @@ __global__ void __launch_bounds__(kQkThreads, 1)
 
 // ======================================================================================
 // pv_softmax: the row softmax and ring pass 2 in one kernel.
-//   P[i][j] = 2^(S[i][j] - m_i) / l_i,   O_i = sum over the ring of P[i][block m] V_m
+//   P[i][j] = 2^(S[i][j] - m_i - log2 l_i),   O_i = sum over the ring of P[i][block m] V_m
 // where (m_i, l_i) combine the per-row partials that qk_slab left (max and sum of 2^(s - max)
 // per 128 key columns), and lse_i = ln 2 (m_i + log2 l_i) is written for the backward pass.
 // Work unit: (128-row tile, head), longest causal tiles first; the key blocks (64 keys) of a
 // unit are visited in ring order from the block of the tile's own chunk. Per step the
 // producer loads the fp32 score block (two 32-column boxes, 128 rows) and the V block; the
-// epilogue warps turn the scores into bf16 P in TMEM (keys 32g .. 32g + 31 of the block in
-// columns 16g .. 16g + 15 of the buffer) and the MMA thread accumulates O += P V with P as
-// the TMEM operand. P never goes back to HBM: the slab is read once, in fp32.
-// Roles (320 threads): warp 0 lane 0 TMA producer, warp 1 TMEM owner and MMA issuer,
-// warps 2..9 epilogue (TMEM lanes 32*(w%4)..+31 = rows; keys 32*((w-2)/4)..+31 of a block).
+// epilogue warps turn the scores into bf16 P in TMEM (key k of the block in column k / 2 of
+// the buffer, two keys per column) and the MMA thread accumulates O += P V with P as the TMEM
+// operand. P never goes back to HBM: the slab is read once, in fp32.
+// Roles: warp 0 lane 0 TMA producer, warp 1 TMEM owner and MMA issuer, then EW epilogue warps:
+// warp w reads TMEM lanes 32*(w%4)..+31 (its rows) and takes KS = 256 / EW keys of each block
+// (slice (w-2)/4). 8 epilogue warps (32 keys each); d = 64: two CTAs per SM (2 stages, 97 KB of
+// shared memory and 256 TMEM columns apiece); d = 128: one CTA per SM with 4 stages. (16
+// epilogue warps of 16 keys at d = 128 were measured slower: twice the barrier hand-offs per
+// block for the same work.)
 // ======================================================================================
-constexpr int kPvThreads = 320;
-constexpr int kPvEpiWarps = 8;
-
 template <int D>
 struct PvCfg {
-    static constexpr int S_BYTES = 128 * 64 * 4;   // [128 rows][64 keys] fp32, two 16 KB boxes
-    static constexpr int V_BYTES = 64 * D * 2;     // [64 keys][D] bf16
+    static constexpr int EW = 8;                      // epilogue warps
+    static constexpr int THREADS = 64 + 32 * EW;
+    static constexpr int KS = 256 / EW;               // keys of a block per epilogue warp
+    static constexpr int OCOLS = D / (EW / 4);        // O columns stored per epilogue warp
+    static constexpr int S_BYTES = 128 * 64 * 4;      // [128 rows][64 keys] fp32, two 16 KB boxes
+    static constexpr int V_BYTES = 64 * D * 2;        // [64 keys][D] bf16
     static constexpr int STAGE_BYTES = S_BYTES + V_BYTES;
-    // d = 64: two CTAs per SM (2 stages each, 97 KB of shared memory and 256 TMEM columns
-    // apiece) so that twice the warps hide the latency of the streaming loads and of the
-    // barrier hand-offs; d = 128 does not fit twice and keeps one CTA with 4 stages
     static constexpr int CTAS = D == 64 ? 2 : 1;
     static constexpr int STAGES = D == 64 ? 2 : 4;
-    static constexpr int OUT_BUFS = 1;                // 2 KB staging buffer per warp
-    static constexpr int OFF_OUT = STAGES * STAGE_BYTES;
-    static constexpr int OFF_CTL = OFF_OUT + kPvEpiWarps * OUT_BUFS * 2048;
+    static constexpr int OFF_OUT = STAGES * STAGE_BYTES;  // 2 KB staging buffer per warp
+    static constexpr int OFF_CTL = OFF_OUT + EW * 2048;
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t T_O = 64;            // P[b] at 32 b (bf16 pairs), O at 64
     static_assert(T_O + D <= TMEM_COLS, "TMEM columns");
+    static_assert(OCOLS % 32 == 0 && KS % 16 == 0, "epilogue slices");
 };
 
 struct PvCtl {
@@ -322,8 +324,24 @@ __device__ __forceinline__ uint32_t pv_sw64(uint32_t row, uint32_t g) {
     return row * 64u + ((g ^ ((row >> 1) & 3u)) << 4);
 }
 
+// P = 2^(s - ml) for the KS scores of one row (16-byte chunks c0 .. c0 + KS/4 - 1 of the row in
+// a 128-byte-swizzled [128 rows][32 keys] fp32 box), as bf16 pairs
+template <int KS>
+__device__ __forceinline__ void pv_probs(const uint8_t *box, uint32_t row, uint32_t c0, float ml,
+                                         uint32_t (&w)[KS / 2]) {
+    const float2 m2 = make_float2(ml, ml);
+#pragma unroll
+    for (int c = 0; c < KS / 4; ++c) {
+        const float4 x = *reinterpret_cast<const float4 *>(box + sw128_offset(row, c0 + c));
+        const float2 lo = fsub2(make_float2(x.x, x.y), m2);
+        const float2 hi = fsub2(make_float2(x.z, x.w), m2);
+        w[2 * c] = pack_bf16x2(fast_exp2(lo.x), fast_exp2(lo.y));
+        w[2 * c + 1] = pack_bf16x2(fast_exp2(hi.x), fast_exp2(hi.y));
+    }
+}
+
 template <int D>
-__global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
+__global__ void __launch_bounds__(PvCfg<D>::THREADS, PvCfg<D>::CTAS)
     pv_softmax_kernel(const __grid_constant__ CUtensorMap mS, const __grid_constant__ CUtensorMap mV,
                       const __grid_constant__ CUtensorMap mO, float *__restrict__ lse,
                       const SlabArgs a) {
@@ -339,11 +357,11 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
             mbar_init(&ctl->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&ctl->pready[b], kPvEpiWarps);
+            mbar_init(&ctl->pready[b], C::EW);
             mbar_init(&ctl->pfree[b], 1);
         }
         mbar_init(&ctl->accfull, 1);
-        mbar_init(&ctl->accempty, kPvEpiWarps);
+        mbar_init(&ctl->accempty, C::EW);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
@@ -437,11 +455,13 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
+        const int ew = warp - 2, q = warp & 3, ks = ew >> 2;  // ks: this warp's key slice
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-        uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
+        uint8_t *obuf = smem + C::OFF_OUT + ew * 2048;
+        // the slice's keys in the score block: box (ks * KS) / 32, 16-byte chunks from c0
+        const int kbox = (ks * C::KS) / 32;
+        const uint32_t c0 = ((ks * C::KS) % 32) / 4;
         uint32_t gstep = 0, acc_ph = 0;
-        int obuf = 0;
         Pipe p{0, 0};
         bool ok = true;
         for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
@@ -451,7 +471,7 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
             const int iw = tl.i0 + 32 * q;  // this warp's first row
             const int i = iw + lane;         // this thread's row
             // the row's softmax statistics from the slab GEMM's partials
-            float m = 0.f, inv = 0.f;
+            float ml = 0.f;
             if (i < a.r0 + a.R) {
                 // causal: the partials of the windows up to the one holding the tile's last
                 // live key (each window holds 2 * ceil(wlen / 256) slots)
@@ -462,16 +482,14 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                     nlive = wl * 2 * ((a.wlen + 255) / 256) + 2 * ((end - wl * a.wlen + 255) / 256);
                 }
                 const float2 *st = a.stats + (static_cast<size_t>(tl.h) * a.R + (i - a.r0)) * a.nStat;
-                float l = 0.f;
-                m = -INFINITY;
+                float m = -INFINITY, l = 0.f;
                 for (int k = 0; k < nlive; ++k) {
                     const float2 x = st[k];
                     softmax_combine(m, l, x.x, x.y);
                 }
-                inv = 1.f / l;
-                if (hf == 0)
-                    lse[static_cast<size_t>(bh) * a.Lq + (i - a.qrow0)] =
-                        (m + __log2f(l)) * 0.6931471805599453f;
+                ml = m + __log2f(l);
+                if (ks == 0)
+                    lse[static_cast<size_t>(bh) * a.Lq + (i - a.qrow0)] = ml * 0.6931471805599453f;
             }
             for (int s = 0; s < tl.nkb; ++s) {
                 const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
@@ -481,16 +499,15 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                     ok = false;
                     break;
                 }
-                const uint8_t *sb = smem + p.stage * C::STAGE_BYTES + hf * 16384;
-                uint32_t w[16];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sb + sw128_offset(32 * q + lane, c));
-                    w[2 * c] = pack_bf16x2(fast_exp2(x.x - m) * inv, fast_exp2(x.y - m) * inv);
-                    w[2 * c + 1] = pack_bf16x2(fast_exp2(x.z - m) * inv, fast_exp2(x.w - m) * inv);
-                }
+                const uint8_t *box = smem + p.stage * C::STAGE_BYTES + kbox * 16384;
+                uint32_t w[C::KS / 2];
+                pv_probs<C::KS>(box, 32 * q + lane, c0, ml, w);
                 tc_fence_after();
-                tmem_st16(tmem + lane_base + 32 * b + 16 * hf, w);
+                const uint32_t tcol = tmem + lane_base + 32 * b + (ks * C::KS) / 2;
+                if constexpr (C::KS == 32)
+                    tmem_st16(tcol, w);
+                else
+                    tmem_st8(tcol, w);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -499,24 +516,22 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                 ++gstep;
             }
             if (!ok) break;
-            // O of this tile, bf16, through the staging buffer
+            // O of this tile, bf16, through the staging buffer: OCOLS columns per warp
             if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
             acc_ph ^= 1u;
             tc_fence_after();
-            uint32_t r[D / 64][32];
+            uint32_t r[C::OCOLS / 32][32];
 #pragma unroll
-            for (int cc = 0; cc < D / 64; ++cc)
-                tmem_ld32(tmem + lane_base + C::T_O + hf * (D / 2) + 32 * cc, r[cc]);
+            for (int cc = 0; cc < C::OCOLS / 32; ++cc)
+                tmem_ld32(tmem + lane_base + C::T_O + ks * C::OCOLS + 32 * cc, r[cc]);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->accempty);
             if (iw >= a.r0 + a.R) continue;  // the whole 32-row box lies past the group's rows
 #pragma unroll
-            for (int cc = 0; cc < D / 64; ++cc) {
-                uint8_t *buf = obase + obuf * 2048;
-                obuf = obuf + 1 == C::OUT_BUFS ? 0 : obuf + 1;
-                if (lane == 0) bulk_wait_read<C::OUT_BUFS - 1>();
+            for (int cc = 0; cc < C::OCOLS / 32; ++cc) {
+                if (lane == 0) bulk_wait_read<0>();
                 __syncwarp();
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -525,12 +540,12 @@ __global__ void __launch_bounds__(kPvThreads, PvCfg<D>::CTAS)
                     for (int u = 0; u < 4; ++u)
                         v[u] = pack_bf16x2(__uint_as_float(r[cc][8 * g + 2 * u]),
                                            __uint_as_float(r[cc][8 * g + 2 * u + 1]));
-                    *reinterpret_cast<uint4 *>(buf + pv_sw64(lane, g)) = make_uint4(v[0], v[1], v[2], v[3]);
+                    *reinterpret_cast<uint4 *>(obuf + pv_sw64(lane, g)) = make_uint4(v[0], v[1], v[2], v[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mO, buf, hf * (D / 2) + 32 * cc, iw - a.qrow0, bh);
+                    tma_store_3d(&mO, obuf, ks * C::OCOLS + 32 * cc, iw - a.qrow0, bh);
                     bulk_commit();
                 }
             }
@@ -582,10 +597,10 @@ cudaError_t launch_pv_softmax(const CUtensorMap &mS, const CUtensorMap &mV, cons
                               float *lse, const SlabArgs &a, int num_sms, cudaStream_t st) {
     const int grid = tc::grid_for(a.ntiles, num_sms * (a.d == 64 ? PvCfg<64>::CTAS : PvCfg<128>::CTAS));
     if (a.d == 64)
-        return launch_pdl(pv_softmax_kernel<64>, dim3(grid), dim3(kPvThreads), pv_smem<64>(), st,
-                          mS, mV, mO, lse, a);
-    return launch_pdl(pv_softmax_kernel<128>, dim3(grid), dim3(kPvThreads), pv_smem<128>(), st,
-                      mS, mV, mO, lse, a);
+        return launch_pdl(pv_softmax_kernel<64>, dim3(grid), dim3(PvCfg<64>::THREADS), pv_smem<64>(),
+                          st, mS, mV, mO, lse, a);
+    return launch_pdl(pv_softmax_kernel<128>, dim3(grid), dim3(PvCfg<128>::THREADS), pv_smem<128>(),
+                      st, mS, mV, mO, lse, a);
 }
 
 }  // namespace rsa

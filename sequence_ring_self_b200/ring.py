@@ -215,7 +215,7 @@ def run_lockstep(gens):
 
 class Kernels:
     """The per-rank steps through the library's C ABI (include/rsa_sp.h), bf16 on one GPU.
-    Workspaces are allocated once per shape and reused by every step."""
+    Workspaces are allocated once per rank state and shape and reused by every step."""
 
     def __init__(self):
         self.lib = rsa.load_library()
@@ -240,8 +240,10 @@ class Kernels:
         return B, H, c * P, d
 
     def _workspace(self, st, P, bwd):
+        """The rank's own workspace (its score slab, its rows' statistics): one per rank state,
+        so that the ranks of an emulated ring never share one."""
         B, H, L, d = self._dims(st, P)
-        key = (B, H, L, d, P, bool(st.causal), bwd, st.q.device)
+        key = (id(st), B, H, L, d, P, bool(st.causal), bwd, st.q.device)
         if key not in self._ws:
             n = self.lib.rsa_sp_workspace_size(B, H, L, d, P, int(st.causal), int(bwd))
             if n == 0:

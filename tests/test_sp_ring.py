@@ -255,6 +255,8 @@ SP_GPU = [  # (B, H, L, d, P)
     (1, 4, 2048, 64, 8),
     (1, 2, 768, 128, 3),   # chunk of 256 keys: window tiles end exactly at the chunk's end
     (1, 2, 384, 64, 3),    # chunk of 128 keys: a 256-key tile reaches past the window
+    (1, 2, 512, 64, 4, "unscaled"),   # score std ~1: wrong scores or statistics would show
+    (1, 2, 768, 128, 3, "unscaled"),
 ]
 
 
@@ -269,8 +271,10 @@ def test_gpu_ring_kernels_match_the_oracle(orc, shape, causal):
     build.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    B, H, L, d, P = shape
-    x = make_inputs(B, H, L, d, seed=800 + L + P, dtype="bf16")
+    B, H, L, d, P = shape[:5]
+    unscaled = len(shape) > 5
+    x = make_inputs(B, H, L, d, seed=800 + L + P, dtype="bf16",
+                    qkv_scale=1.0 if unscaled else None)
     got = _lockstep(x, P, causal, ring.Kernels(), get=lambda n: x.torch(n, dev))
     torch.cuda.synchronize()
     assert rsa.last_device_status() == rsa.RSA_OK
@@ -279,14 +283,22 @@ def test_gpu_ring_kernels_match_the_oracle(orc, shape, causal):
     for n, ref in refs.items():
         err = np.abs(got[n] - ref).max()
         rel = np.linalg.norm(got[n] - ref) / np.linalg.norm(ref)
-        assert err <= BF16_MAXABS and rel <= BF16_RELL2, (n, err, rel)
-    np.testing.assert_allclose(got["lse"], lse, rtol=0, atol=1e-3)
+        # unscaled inputs give outputs beyond 8 (one bf16 ulp 0.0625): max-abs relative to the
+        # tensor's largest magnitude, as in the single-device sharp-attention cases
+        bound = BF16_MAXABS * (max(1.0, float(np.abs(ref).max())) if unscaled else 1.0)
+        assert err <= bound and rel <= BF16_RELL2, (n, err, rel)
+    np.testing.assert_allclose(got["lse"], lse, rtol=1e-3 if unscaled else 0, atol=1e-3)
     # against the single-device path on the same inputs
     q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
     o1, lse1 = rsa.forward(q, k, v, P, causal)
     dq1, dk1, dv1 = rsa.backward(q, k, v, o1, do, lse1, P, causal)
-    np.testing.assert_allclose(got["lse"], lse1.cpu().numpy(), rtol=0, atol=1e-5)
+    np.testing.assert_allclose(got["lse"], lse1.cpu().numpy(), rtol=1e-5, atol=1e-5)
+    # both paths are within the bf16 bound of the oracle (checked above), so they are within
+    # twice that bound of each other (two bf16 roundings can differ by a whole ulp, 0.03125
+    # for values in [4, 8))
     for n, t in (("o", o1), ("dq", dq1), ("dk", dk1), ("dv", dv1)):
         ref = t.to("cpu", torch.float64).numpy()
         err = np.abs(got[n] - ref).max()
-        assert err <= BF16_MAXABS, (n, err)
+        rel = np.linalg.norm(got[n] - ref) / np.linalg.norm(ref)
+        bound = 2 * BF16_MAXABS * (max(1.0, float(np.abs(ref).max())) if unscaled else 1.0)
+        assert err <= bound and rel <= 2 * BF16_RELL2, (n, err, rel)
