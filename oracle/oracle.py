@@ -51,6 +51,7 @@ _SIGS = {
     "rsa_oracle_forward_rows": [_D, _D, _D, _l, _l, _i, _LP, _l, _D, _D],
     "rsa_oracle_backward_rows": [_D, _D, _D, _D, _l, _l, _i, _LP, _l, _D],
     "rsa_oracle_backward_keys": [_D, _D, _D, _D, _l, _l, _i, _LP, _l, _D, _D],
+    "rsa_oracle_linear": [_D, _D, _D, _D, _l, _l, _l, _i, _D],
 }
 
 
@@ -202,6 +203,27 @@ def backward_keys(q, k, v, do, b: int, h: int, keys, causal: bool = False):
                                             int(causal), r.ctypes.data_as(_LP), len(r), _ptr(dk),
                                             _ptr(dv)), "backward_keys")
     return dk, dv
+
+
+def linear(x, w, b=None, r=None, gelu: bool = False):
+    """Y = act(X W^T + b) + R on rows: X [M, K], W [N, K], b [N] or None, R [M, N] or None;
+    act = exact GELU when `gelu`, else the identity. Returns Y [M, N] fp64."""
+    x, w = _f64(x), _f64(w)
+    if x.ndim != 2 or w.ndim != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("expected X [M, K] and W [N, K]")
+    M, K = x.shape
+    N = w.shape[0]
+    bb = _f64(b) if b is not None else None
+    rr = _f64(r) if r is not None else None
+    if bb is not None and bb.shape != (N,):
+        raise ValueError("bias must be [N]")
+    if rr is not None and rr.shape != (M, N):
+        raise ValueError("residual must be [M, N]")
+    y = np.empty((M, N))
+    _check(_load().rsa_oracle_linear(_ptr(x), _ptr(w), _ptr(bb) if bb is not None else None,
+                                     _ptr(rr) if rr is not None else None, M, N, K, int(gelu),
+                                     _ptr(y)), "linear")
+    return y
 
 
 @contextlib.contextmanager

@@ -508,3 +508,35 @@ int rsa_oracle_backward_keys(const double *Qh, const double *Kh, const double *V
     free(Dv);
     return err;
 }
+
+/* ------------------------------------------------------------------ linear layers of the block
+ *
+ * Sequence parallelism splits the whole Transformer block, not only its attention, by the
+ * sequence (review page, Abstract: every device holds a chunk of the sequence; the layers
+ * other than self-attention work on their own chunk's rows with no exchange). The block's
+ * linear layers (the query/key/value projection, the output projection and the two layers of
+ * the MLP) are, on a chunk of M rows,
+ *
+ *   Y[m][n] = act( sum_k X[m][k] W[n][k] + b[n] ) + R[m][n]
+ *
+ * with W [N][K] (out x in), an optional bias b [N] (NULL: none), an optional residual R [M][N]
+ * (NULL: none) and act the identity or, when gelu != 0, the exact GELU
+ *   GELU(x) = x Phi(x) = x (1 + erf(x / sqrt 2)) / 2
+ * (Phi the standard normal distribution function). Row-major fp64 throughout.
+ */
+int rsa_oracle_linear(const double *X, const double *W, const double *b, const double *R, long M,
+                      long N, long K, int gelu, double *Y) {
+    if (!X || !W || !Y || M <= 0 || N <= 0 || K <= 0) return -1;
+#pragma omp parallel for schedule(static)
+    for (long m = 0; m < M; ++m) {
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k) acc += X[m * K + k] * W[n * K + k];
+            if (b) acc += b[n];
+            if (gelu) acc = 0.5 * acc * (1.0 + erf(acc / sqrt(2.0)));
+            if (R) acc += R[m * N + n];
+            Y[m * N + n] = acc;
+        }
+    }
+    return 0;
+}

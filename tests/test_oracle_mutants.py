@@ -33,6 +33,14 @@ MUTANTS = {
     "ring wrong key block": ("acc += S[ii * L + m * c + jj] * Vh[(m * c + jj) * d + k];",
                              "acc += S[ii * L + m * c + jj] * Vh[(n * c + jj) * d + k];"),
     "ring dV wrong row": ("dVh[j * d + k] += p * dOh[i * d + k];", "dVh[j * d + k] += p * dOh[j * d + k];"),
+    "linear bias dropped": ("            if (b) acc += b[n];\n", ""),
+    "GELU half dropped": ("if (gelu) acc = 0.5 * acc * (1.0 + erf(acc / sqrt(2.0)));",
+                          "if (gelu) acc = acc * (1.0 + erf(acc / sqrt(2.0)));"),
+    "residual inside the GELU": (
+        "            if (gelu) acc = 0.5 * acc * (1.0 + erf(acc / sqrt(2.0)));\n            if (R) acc += R[m * N + n];",
+        "            if (R) acc += R[m * N + n];\n            if (gelu) acc = 0.5 * acc * (1.0 + erf(acc / sqrt(2.0)));"),
+    "linear weight row/column swapped": ("acc += X[m * K + k] * W[n * K + k];",
+                                         "acc += X[m * K + k] * W[(k % N) * K + (n % K)];"),
 }
 
 
@@ -49,6 +57,9 @@ def _battery(orc):
         ("finite differences", lambda: pins.test_backward_matches_finite_differences(orc, 5, 3, False)),
         ("finite differences causal", lambda: pins.test_backward_matches_finite_differences(orc, 5, 3, True)),
         ("invariants", lambda: pins.test_backward_invariants(orc, False)),
+        ("linear", lambda: pins.test_linear_matches_plain_python(orc, False, True, False)),
+        ("linear gelu residual", lambda: pins.test_linear_matches_plain_python(orc, True, True, True)),
+        ("gelu values", lambda: pins.test_gelu_values_and_symmetry(orc)),
     ]
     failed = []
     for name, fn in checks:

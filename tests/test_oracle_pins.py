@@ -276,3 +276,60 @@ def test_sampled_rows_and_keys_match_full(orc, causal):
     dkr, dvr = orc.backward_keys(x.q, x.k, x.v, x.do, 0, 1, rows, causal)
     np.testing.assert_allclose(dkr, dk[0, 1, rows], rtol=1e-11, atol=1e-15)
     np.testing.assert_allclose(dvr, dv[0, 1, rows], rtol=1e-11, atol=1e-15)
+
+
+# ------------------------------------------------------------------ linear layers of the block
+
+def _py_linear(x, w, b, r, gelu):
+    """The definition in plain Python floats (math.fsum, math.erf): an independent restatement."""
+    M, K = len(x), len(x[0])
+    N = len(w)
+    y = []
+    for m in range(M):
+        row = []
+        for n in range(N):
+            acc = math.fsum(x[m][k] * w[n][k] for k in range(K)) + (b[n] if b is not None else 0.0)
+            if gelu:
+                acc = 0.5 * acc * (1.0 + math.erf(acc / math.sqrt(2.0)))
+            row.append(acc + (r[m][n] if r is not None else 0.0))
+        y.append(row)
+    return np.array(y)
+
+
+@pytest.mark.parametrize("gelu", [False, True])
+@pytest.mark.parametrize("with_bias,with_res", [(False, False), (True, False), (True, True)])
+def test_linear_matches_plain_python(orc, gelu, with_bias, with_res):
+    rng = np.random.default_rng(31)
+    M, N, K = 3, 5, 7
+    x, w = rng.normal(size=(M, K)), rng.normal(size=(N, K))
+    b = rng.normal(size=N) if with_bias else None
+    r = rng.normal(size=(M, N)) if with_res else None
+    got = orc.linear(x, w, b, r, gelu)
+    ref = _py_linear(x.tolist(), w.tolist(), None if b is None else b.tolist(),
+                     None if r is None else r.tolist(), gelu)
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_gelu_values_and_symmetry(orc):
+    """GELU(x) = x Phi(x): GELU(0) = 0, GELU(x) - GELU(-x) = x (Phi(x) + Phi(-x) = 1),
+    GELU(1) = Phi(1) = 0.8413447460685429 (the standard normal CDF at 1), GELU(10) = 10 and
+    GELU(-10) = 0 to double precision."""
+    xs = np.array([[0.0, 1.0, -1.0, 2.5, -2.5, 10.0, -10.0]])
+    eye = np.eye(1)
+    y = orc.linear(xs.T, eye, gelu=True)[:, 0]
+    assert y[0] == 0.0
+    assert y[1] == pytest.approx(0.8413447460685429, abs=1e-15)
+    assert y[1] - y[2] == pytest.approx(1.0, abs=1e-15)
+    assert y[3] - y[4] == pytest.approx(2.5, abs=1e-15)
+    assert y[5] == pytest.approx(10.0, abs=1e-14) and abs(y[6]) < 1e-20
+
+
+def test_linear_identity_weight_and_residual(orc):
+    rng = np.random.default_rng(32)
+    x, r = rng.normal(size=(4, 6)), rng.normal(size=(4, 6))
+    np.testing.assert_array_equal(orc.linear(x, np.eye(6)), x)
+    np.testing.assert_allclose(orc.linear(x, np.eye(6), r=r), x + r, rtol=0, atol=1e-15)
+    # the bias adds to every row; the weight is used as out x in (a transposed weight fails)
+    w = rng.normal(size=(3, 6))
+    b = rng.normal(size=3)
+    np.testing.assert_allclose(orc.linear(x, w, b), x @ w.T + b, rtol=1e-13, atol=1e-13)
