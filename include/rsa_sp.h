@@ -89,6 +89,27 @@ RSA_API rsa_status_t rsa_sp_backward_keys(const void *Q, const void *Kfull, cons
 RSA_API rsa_status_t rsa_sp_accumulate(float *acc, const void *part, void *out, long long n,
                                        int first, void *stream);
 
+/*
+ * The block's linear layers on a rank's rows (the rest of the block needs no exchange under
+ * sequence parallelism: review page, Abstract). On M rows:
+ *
+ *   Y[m][n] = act( sum_k X[m][k] W[n][k] + bias[n] ) + R[m][n]
+ *
+ * act = exact GELU (x Phi(x)) when gelu != 0, else the identity. bf16 operands, fp32
+ * accumulation on the tensor cores, bf16 output rounded to nearest-even.
+ * X: bf16, the row-major [M][K] matrix stored as [K / x_kin][M][x_kin] (x_kin = K: a plain
+ *    row-major X; x_kin = d: the [H][M][d] output of attention, read as [M][H d]).
+ * W: bf16 [N][K] row-major (out x in). bias: fp32 [N] or NULL. R: bf16 [M][N] or NULL
+ *    (residual; only with y_kin == N).
+ * Y: bf16, the [M][N] result stored as [N / y_kin][M][y_kin] (y_kin = N: plain; y_kin = d: the
+ *    query/key/value projection written straight into [3 H][M][d] for attention).
+ * Supported: M % 128 == 0, N % 64 == 0, K % 64 == 0, x_kin % 64 == 0 dividing K, y_kin % 32 ==
+ * 0 dividing N; RSA_ERR_UNSUPPORTED otherwise. Pointers 16-byte aligned. Errors as in rsa.h.
+ */
+RSA_API rsa_status_t rsa_linear(const void *X, const void *W, const float *bias, const void *R,
+                                void *Y, int M, int N, int K, int x_kin, int y_kin, int gelu,
+                                void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -259,7 +259,8 @@ rsa_status_t device_state(DeviceState **out) {
         if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
         if ((e = rsa::tc_kernels_configure()) != cudaSuccess ||
             (e = rsa::bwd_kernels_configure()) != cudaSuccess ||
-            (e = rsa::fwd_kernels_configure()) != cudaSuccess)
+            (e = rsa::fwd_kernels_configure()) != cudaSuccess ||
+            (e = rsa::linear_kernels_configure()) != cudaSuccess)
             return cuda_fail("cudaFuncSetAttribute", e);
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, rsa::g_status_word);
@@ -284,12 +285,12 @@ rsa_status_t device_state(DeviceState **out) {
 
 enum Kind {
     K_QK_SLAB, K_SOFTMAX, K_PV, K_ROWDOT, K_BWD_KEYS, K_BWD_ROWS,
-    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_FWD_STATS, K_FWD_PV, K_SP_ACC, K_COUNT
+    K_F32_QK, K_F32_PV, K_F32_BWD, K_F32_KEYS, K_F32_DQ, K_FWD_STATS, K_FWD_PV, K_SP_ACC, K_LINEAR, K_COUNT
 };
 const char *kKindNames[K_COUNT] = {
     "qk_slab", "slab_softmax", "pv_softmax", "rowdot", "bwd_keys", "bwd_rows",
     "f32_qk_slab", "f32_pv_ring_rows", "f32_bwd_slab", "f32_ring_keys", "f32_dq_ring_rows",
-    "fwd_stats", "fwd_pv", "sp_accumulate"};
+    "fwd_stats", "fwd_pv", "sp_accumulate", "linear"};
 
 struct ProfRec {
     int kind;
@@ -947,6 +948,39 @@ rsa_status_t rsa_sp_accumulate(float *acc, const void *part, void *out, long lon
                               acc, static_cast<const __nv_bfloat16 *>(part),
                               static_cast<__nv_bfloat16 *>(out), n, first ? 1 : 0),
                           cudaGetLastError()));
+    return RSA_OK;
+}
+
+rsa_status_t rsa_linear(const void *X, const void *W, const float *bias, const void *R, void *Y,
+                        int M, int N, int K, int x_kin, int y_kin, int gelu, void *stream) {
+    if (!X || !W || !Y || !aligned16(X) || !aligned16(W) || !aligned16(Y) ||
+        (bias && !aligned16(bias)) || (R && !aligned16(R)))
+        return RSA_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || x_kin <= 0 || y_kin <= 0) return RSA_ERR_INVALID_ARG;
+    if (M % 128 != 0 || N % 64 != 0 || K % 64 != 0 || x_kin % 64 != 0 || K % x_kin != 0 ||
+        y_kin % 32 != 0 || N % y_kin != 0 || (R && y_kin != N))
+        return RSA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(M / 128) * ((N + 255) / 256) > 0x3fffffffLL) return RSA_ERR_UNSUPPORTED;
+    DeviceState *dev = nullptr;
+    rsa_status_t st = device_state(&dev);
+    if (st != RSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUtensorMap mX, mW, mY;
+    if (!map3d(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, x_kin, M, K / x_kin, uint64_t(x_kin) * 2,
+               uint64_t(M) * x_kin * 2, 64, 128) ||
+        !map3d(&mW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, K, N, 1, uint64_t(K) * 2,
+               uint64_t(N) * K * 2, 64, 256) ||
+        !map3d(&mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, y_kin, M, N / y_kin, uint64_t(y_kin) * 2,
+               uint64_t(M) * y_kin * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return RSA_ERR_CUDA;
+    rsa::LinArgs a{};
+    a.M = M, a.N = N, a.K = K, a.x_kin = x_kin, a.y_kin = y_kin, a.gelu = gelu ? 1 : 0;
+    a.bias = bias;
+    a.res = static_cast<const __nv_bfloat16 *>(R);
+    a.nNT = (N + 255) / 256;
+    a.ntiles = (M / 128) * a.nNT;
+    a.status = dev->status;
+    RSA_LAUNCH(K_LINEAR, rsa::launch_linear(mX, mW, mY, a, dev->sms, s));
     return RSA_OK;
 }
 

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -109,6 +110,22 @@ cudaError_t launch_fwd_pv(const CUtensorMap &mQ, const CUtensorMap &mK, const CU
 cudaError_t fwd_kernels_configure();
 cudaError_t tc_kernels_configure();  // opt-in shared memory sizes (once per device)
 cudaError_t bwd_kernels_configure();
+
+// ---- the block's linear layers (kernels_linear.cu) ----------------------------------------
+// Y = act(X W^T + b) + R on M rows. X is read as (x_kin, M, K / x_kin) and Y written as
+// (y_kin, M, N / y_kin) bf16 tensors (a plain row-major matrix has x_kin = K / y_kin = N).
+struct LinArgs {
+    int M, N, K;
+    int x_kin, y_kin;
+    int gelu;
+    const float *bias;           // [N] or null
+    const __nv_bfloat16 *res;    // [M][N] row-major or null
+    int ntiles, nNT;             // (M / 128) x ceil(N / 256) tiles; nNT = ceil(N / 256)
+    int *status;
+};
+cudaError_t launch_linear(const CUtensorMap &mX, const CUtensorMap &mW, const CUtensorMap &mY,
+                          const LinArgs &a, int num_sms, cudaStream_t st);
+cudaError_t linear_kernels_configure();
 
 // ---- CUDA-core kernels (kernels_simt.cu) -----------------------------------------------
 // Row softmax of the group's fp32 slab, in place: P written as bf16 (p_bf16 = 1) into the

@@ -28,7 +28,10 @@ EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_str
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
             "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
             "rsa_forward_noalloc", "rsa_last_error", "rsa_forward_recompute",
-            "rsa_probe_ffma", "rsa_probe_ffma_flops_per_thread", "rsa_debug_report_status")
+            "rsa_probe_ffma", "rsa_probe_ffma_flops_per_thread", "rsa_debug_report_status",
+            # include/rsa_sp.h
+            "rsa_sp_workspace_size", "rsa_sp_scores", "rsa_sp_softmax_pv", "rsa_sp_backward_rows",
+            "rsa_sp_backward_keys", "rsa_sp_accumulate", "rsa_linear")
 
 _lib = None
 _lock = threading.Lock()
@@ -91,6 +94,8 @@ def load_library(path: str | None = None):
         lib.rsa_probe_ffma_flops_per_thread.restype = ctypes.c_longlong
         lib.rsa_debug_report_status.argtypes = [i, vp]
         lib.rsa_debug_report_status.restype = i
+        lib.rsa_linear.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+        lib.rsa_linear.restype = i
         if path is None:
             _lib = lib
         return lib
@@ -330,3 +335,47 @@ def forward_backward_host(q, k, v, do, N: int, causal: bool = False, *, ws_budge
     for n, t in zip(names, (o, lse, dq, dk, dv)):
         results[n].copy_(t, non_blocking=True)
     return results
+
+
+def linear(x, w, bias=None, residual=None, gelu: bool = False, *, x_kin: int | None = None,
+           y_kin: int | None = None, out=None, stream: torch.cuda.Stream | None = None):
+    """Y = act(X W^T + bias) + residual on M rows (include/rsa_sp.h, rsa_linear), bf16.
+
+    x: [M, K] bf16, or (x_kin = d) the [H, M, d] output of attention read as [M, H d];
+    w: [N, K] bf16; bias: [N] fp32 or None; residual: [M, N] bf16 or None.
+    Returns Y [M, N], or with y_kin = d the [N / d, M, d] layout (the query/key/value
+    projection written for attention)."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("linear takes bf16 X and W")
+    if not (x.is_contiguous() and w.is_contiguous()):
+        raise ValueError("X and W must be contiguous")
+    N, K = w.shape
+    if x.dim() == 2:
+        M = x.shape[0]
+        xk = K if x_kin is None else x_kin
+        if x.shape[1] != K or xk != K:
+            raise ValueError("X [M, K] must match W [N, K]")
+    elif x.dim() == 3:
+        M = x.shape[1]
+        xk = x.shape[2]
+        if x_kin not in (None, xk) or x.shape[0] * xk != K:
+            raise ValueError("X [H, M, d] must have H d = K")
+    else:
+        raise ValueError("X must be [M, K] or [H, M, d]")
+    yk = N if y_kin is None else y_kin
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (N,)):
+        raise ValueError("bias must be fp32 [N]")
+    if residual is not None and (residual.dtype != torch.bfloat16 or tuple(residual.shape) != (M, N)
+                                 or not residual.is_contiguous()):
+        raise ValueError("residual must be contiguous bf16 [M, N]")
+    _same_device(x.device, w, bias, residual, out)
+    shape = (M, N) if yk == N else (N // yk, M, yk)
+    with torch.cuda.device(x.device):
+        y = torch.empty(shape, dtype=torch.bfloat16, device=x.device) if out is None else out
+        s = stream if stream is not None else torch.cuda.current_stream(x.device)
+        rc = load_library().rsa_linear(_ptr(x), _ptr(w), _ptr(bias) if bias is not None else None,
+                                       _ptr(residual) if residual is not None else None, _ptr(y),
+                                       M, N, K, xk, yk, int(bool(gelu)), ctypes.c_void_p(s.cuda_stream))
+    if rc != RSA_OK:
+        raise RSAError(rc, "rsa_linear")
+    return y

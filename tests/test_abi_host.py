@@ -19,8 +19,12 @@ def lib():
 
 
 def _declared():
-    text = open(os.path.join(ROOT, "include", "rsa.h")).read()
-    return re.findall(r"RSA_API\s+[\w\s\*]+?\b(rsa_\w+)\s*\(", text)
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"RSA_API\s+[\w\s\*]+?\b(rsa_\w+)\s*\(", text)
+    return names
 
 
 def test_header_declares_the_abi():
@@ -196,3 +200,18 @@ def test_bindings_refuse_outputs_on_another_device():
     cpu = torch.empty(4)
     with pytest.raises(ValueError, match="expected cuda:0"):
         rsa._same_device(torch.device("cuda", 0), None, cpu)
+
+
+def _lin(lib, M=128, N=64, K=64, xk=64, yk=64, ptr=FAKE, res=None, bias=None):
+    return lib.rsa_linear(ptr, ptr, bias, res, ptr, M, N, K, xk, yk, 0, None)
+
+
+def test_linear_argument_errors(lib):
+    assert _lin(lib, ptr=0) == rsa.RSA_ERR_INVALID_ARG
+    assert _lin(lib, ptr=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG
+    assert _lin(lib, M=0) == rsa.RSA_ERR_INVALID_ARG
+    assert _lin(lib, M=100) == rsa.RSA_ERR_UNSUPPORTED            # rows not a multiple of 128
+    assert _lin(lib, N=96, yk=96) == rsa.RSA_ERR_UNSUPPORTED      # N not a multiple of 64
+    assert _lin(lib, K=96, xk=96) == rsa.RSA_ERR_UNSUPPORTED      # K not a multiple of 64
+    assert _lin(lib, K=256, xk=96) == rsa.RSA_ERR_UNSUPPORTED     # head width not dividing K
+    assert _lin(lib, N=128, yk=64, res=FAKE) == rsa.RSA_ERR_UNSUPPORTED  # residual, split output
