@@ -70,11 +70,13 @@ typedef enum { RSA_F32 = 0, RSA_BF16 = 1 } rsa_dtype_t;
  * The score slab (the c x L block of scores of every chunk, i.e. L x L per head) is
  * processed in groups, one after the other in the same workspace: a group is a set of whole
  * heads, or, when a head does not fit, the same range of rows (a multiple of 128) of one or
- * several heads. On the bf16 forward the groups are balanced: equal rectangles of heads x rows
- * chosen so that no group is a small remainder that would leave most of the GPU idle.
+ * several heads. On the bf16 forward the groups are rectangles of heads x 128-row tiles chosen
+ * to fill whole rounds of the GPU's SMs: the softmax / ring-pass-2 kernel runs one unit
+ * (head, 128-row tile) per CTA, so a group takes ceil(units / resident CTAs) rounds and the
+ * plan takes the rectangles with the fewest rounds in total.
  * `budget_bytes` caps the workspace: the returned size is that of the plan chosen within the
  * budget (or of the smallest plan, one 128-row range of one head, if nothing fits).
- * budget_bytes == 0 asks for the default plan (at most 1 GiB).
+ * budget_bytes == 0 asks for the default plan (at most 4 GiB).
  * for_backward selects the backward call's needs: on the bf16 path the backward keeps no
  * slab (every score tile is recomputed on the chip) and needs only the padded per-row
  * statistics, 8 * B * H * roundup(L, 64) bytes, whatever the budget; the fp32 path keeps fp32

@@ -30,7 +30,7 @@ using rsa::Group;
 using rsa::SlabArgs;
 
 constexpr size_t kAlign = 256;
-constexpr size_t kDefaultBudget = size_t(1) << 30;
+constexpr size_t kDefaultBudget = size_t(4) << 30;
 constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -90,15 +90,18 @@ bool args_ok(int B, int H, int L, int d, int N, rsa_dtype_t dt, rsa_status_t *wh
     return true;
 }
 
-// Work units a slab group should hold for its two kernels to keep HBM busy: a group with fewer
-// (128-row tile, head) units runs about as long as one with this many, since each unit streams
-// its scores at the rate of one SM.
-constexpr long long kSaturatingUnits = 96;
+// The softmax / ring-pass-2 kernel runs a slab group's (head, 128-row tile) units on one CTA
+// each, all units of a group alike in length (each streams its rows' scores), so a group takes
+// about ceil(units / slots) rounds of one unit's time, slots being the CTAs the kernel keeps
+// resident: 148 SMs (B200) times its CTAs per SM (2 at d = 64, 1 at d = 128). One CTA
+// streams at a small share of HBM's bandwidth (measured about 40 GB/s), so a round with few
+// units leaves HBM idle: a group is costed in whole rounds.
+constexpr long long kSms = 148;
+long long pv_slots(int d) { return kSms * (d == 64 ? 2 : 1); }
 
 // bf16 forward: groups are rectangles of Gh heads x R rows (R = rt * 128, or L). Among the
-// rectangles that fit the budget, take the one whose groups cost least in total, a group
-// costing max(its units, kSaturatingUnits): equal groups, none of them a small tail that would
-// run as long as a full one. Head counts are enumerated by their distinct balanced values.
+// rectangles that fit the budget, take the one whose groups take the fewest rounds in total,
+// then the fewest groups. Head counts are enumerated by their distinct balanced values.
 void plan_rect(Plan &p, size_t budget) {
     const long long nRT = (p.L + 127) / 128;
     const size_t tile_bytes = size_t(128) * p.row_bytes;  // one 128-row tile of one head
@@ -106,28 +109,42 @@ void plan_rect(Plan &p, size_t budget) {
     const long long fit_tiles = static_cast<long long>(budget / tile_bytes);
     const long long fit_heads = static_cast<long long>(budget / head_bytes);
     long long best_cost = -1, best_groups = 0, best_nh = 1, best_rt = 1;
+    const long long slots = pv_slots(p.d);
+    auto rounds = [slots](long long u) { return (u + slots - 1) / slots; };
+    // the plan's total rounds for nh heads x rt tiles per group (the last row group of a head
+    // takes the remaining tiles; `balance` first spreads the tiles evenly over the row groups)
+    auto consider = [&](long long nh, long long rt, bool balance) {
+        const long long ngh = (p.BH + nh - 1) / nh, last_h = p.BH - (ngh - 1) * nh;
+        long long ngt = (nRT + rt - 1) / rt;
+        const long long rt2 = balance ? (nRT + ngt - 1) / ngt : rt;
+        ngt = (nRT + rt2 - 1) / rt2;
+        const long long last_t = nRT - (ngt - 1) * rt2;
+        const long long cost = (ngh - 1) * (ngt - 1) * rounds(nh * rt2) + (ngh - 1) * rounds(nh * last_t) +
+                               (ngt - 1) * rounds(last_h * rt2) + rounds(last_h * last_t);
+        const long long groups = ngh * ngt;
+        if (best_cost < 0 || cost < best_cost || (cost == best_cost && groups < best_groups)) {
+            best_cost = cost;
+            best_groups = groups;
+            best_nh = nh;
+            best_rt = rt2;
+        }
+    };
     for (long long gh = 1; gh <= p.BH;) {
         const long long nh = (p.BH + gh - 1) / gh;  // heads per group with gh head groups
-        long long rt = 0;
+        long long rt_max = 0;
         if (fit_heads >= nh)
-            rt = nRT;
+            rt_max = nRT;
         else if (fit_tiles >= nh)
-            rt = fit_tiles / nh;
-        if (rt > 0) {
-            const long long ngh = (p.BH + nh - 1) / nh, last_h = p.BH - (ngh - 1) * nh;
-            long long ngt = (nRT + rt - 1) / rt;
-            const long long rt2 = (nRT + ngt - 1) / ngt;  // balanced tile count
-            ngt = (nRT + rt2 - 1) / rt2;
-            const long long last_t = nRT - (ngt - 1) * rt2;
-            auto c = [](long long u) { return u > kSaturatingUnits ? u : kSaturatingUnits; };
-            const long long cost = (ngh - 1) * (ngt - 1) * c(nh * rt2) + (ngh - 1) * c(nh * last_t) +
-                                   (ngt - 1) * c(last_h * rt2) + c(last_h * last_t);
-            const long long groups = ngh * ngt;
-            if (best_cost < 0 || cost < best_cost || (cost == best_cost && groups < best_groups)) {
-                best_cost = cost;
-                best_groups = groups;
-                best_nh = nh;
-                best_rt = rt2;
+            rt_max = fit_tiles / nh;
+        if (rt_max > 0) {
+            consider(nh, rt_max, true);
+            // tile counts that make a group a whole number of rounds
+            for (long long k = 1; k <= 64; ++k) {
+                const long long rt = k * slots / nh;
+                if (rt < 1) continue;
+                if (rt >= rt_max) break;
+                consider(nh, rt, false);
+                consider(nh, rt, true);
             }
         }
         if (nh == 1) break;

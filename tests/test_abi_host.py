@@ -148,21 +148,26 @@ def test_plans_fit_their_budget_and_grow_with_it(lib, dtype, bwd):
     assert rsa.plan_describe(B, H, L, d, N, False, dtype, bwd, sizes[0] - 1)["fits"] is False
 
 
-def test_forward_groups_are_balanced(lib):
-    """The bf16 forward's slab groups are equal rectangles of heads x 128-row tiles, not a set of
-    full groups plus a small tail: for the long-sequence shape (a head's slab is 1.09 GB, over
-    the 1 GiB default) every group holds at least 96 of the 2048 (head, row tile) units."""
+def test_forward_groups_fill_whole_rounds(lib):
+    """The bf16 forward's slab groups are rectangles of heads x 128-row tiles that fill whole
+    rounds of the softmax/PV kernel's CTAs (148 SMs, one CTA each at d = 128): for the
+    long-sequence shape (a head's slab is 1.09 GB; the 4 GiB default holds 3.7 heads) the plan
+    takes ceil(2048 / 148) = 14 rounds, the fewest possible, and no group is a remainder of a
+    few units."""
     B, H, L, d, N = 1, 16, 16384, 128, 16
     n = rsa.workspace_size(B, H, L, d, N, False, torch.bfloat16, False, 0)
     info = rsa.plan_describe(B, H, L, d, N, False, torch.bfloat16, False, n)
-    assert info["fits"] and n <= (1 << 30)
+    assert info["fits"] and n <= (4 << 30)
     hg, rows = info["heads_per_group"], info["rows_per_group"]
-    tiles = -(-L // 128)
-    rt = rows // 128
+    tiles, rt = -(-L // 128), rows // 128
+    per_head = -(-L // rows)
+    rounds = 0
     for g in range(info["groups"]):
-        heads = min(hg, B * H - (g // -(-L // rows)) * hg)
-        t = min(rt, tiles - (g % -(-L // rows)) * rt)
+        heads = min(hg, B * H - (g // per_head) * hg)
+        t = min(rt, tiles - (g % per_head) * rt)
         assert heads * t >= 96, (g, heads, t)
+        rounds += -(-heads * t // 148)
+    assert rounds == -(-B * H * tiles // 148) == 14
 
 
 def test_default_plan_is_capped_at_one_gib(lib):

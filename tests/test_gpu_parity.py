@@ -159,8 +159,8 @@ def test_config3_gpt_causal(orc):
 
 
 def test_config4_long_sequence(orc):
-    """B=1 H=16 L=16384 d=128 N=16 bf16, forward slab groups in sequence (1 GiB default
-    workspace): sampled rows and sampled keys of two heads."""
+    """B=1 H=16 L=16384 d=128 N=16 bf16, forward slab groups in sequence (the default
+    workspace holds a fifth of the 17 GB slab): sampled rows and sampled keys of two heads."""
     x = make_inputs(1, 16, 16384, 128, seed=4, dtype="bf16")
     info = rsa.plan_describe(1, 16, 16384, 128, 16, False, torch.bfloat16, False,
                              rsa.workspace_size(1, 16, 16384, 128, 16, False, torch.bfloat16, False))
