@@ -24,10 +24,13 @@ namespace {
 using namespace tc;
 
 // ======================================================================================
-// qk_slab: S[h][i - r0][j] = log2(e) * scale * Q_i . K_j  (fp32 scores in base-2 units;
+// qk_slab: S = log2(e) * scale * Q_i . K_j for row i, key j (fp32 scores in base-2 units;
 // -inf where j >= L or causal j > i), and per row and 128-column half tile the softmax
 // partials (max_j S, sum_j 2^(S - max)) that pv_softmax combines into each row's statistics.
 // Tile = 128 query rows x 256 keys; K-loop over d in blocks of 64 (one 128-byte swizzle row).
+// Slab layout: per (head, 128-row tile) of the group, the key chunks of 32 one after the other,
+// each a contiguous [128 rows][32 keys] block (16 KB), so that ring pass 2 streams whole 16 KB
+// blocks from HBM instead of 128-byte row pieces a slab row apart.
 // 320 threads: producer, MMA, and 8 epilogue warps (2 per TMEM lane quarter, 128 columns each).
 // ======================================================================================
 template <int D>
@@ -226,7 +229,9 @@ __global__ void __launch_bounds__(kQkThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mS, buf, j0 - a.kcol0, tl.i0 - a.r0 + 32 * q, tl.h);
+                    // slab tile (head, row tile) holds [key chunk of 32][128 rows][32 keys]
+                    tma_store_4d(&mS, buf, 0, 32 * q, (j0 - a.kcol0) >> 5,
+                                 tl.h * a.nRT + ((tl.i0 - a.r0) >> 7));
                     bulk_commit();
                 }
             }
@@ -400,8 +405,9 @@ __global__ void __launch_bounds__(PvCfg<D>::THREADS, PvCfg<D>::CTAS)
                     uint8_t *st = smem + p.stage * C::STAGE_BYTES;
                     uint64_t *bar = &ctl->full[p.stage];
                     mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                    tma_load_3d(st, &mS, bar, j0, tl.i0 - a.r0, tl.h);
-                    tma_load_3d(st + 16384, &mS, bar, j0 + 32, tl.i0 - a.r0, tl.h);
+                    const int tile = tl.h * a.nRT + ((tl.i0 - a.r0) >> 7);
+                    tma_load_4d(st, &mS, bar, 0, 0, j0 >> 5, tile);
+                    tma_load_4d(st + 16384, &mS, bar, 0, 0, (j0 >> 5) + 1, tile);
 #pragma unroll
                     for (int dp = 0; dp < D / 64; ++dp)
                         tma_load_3d(st + C::S_BYTES + dp * 8192, &mV, bar, dp * 64, j0,

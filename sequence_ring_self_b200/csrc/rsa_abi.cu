@@ -105,7 +105,7 @@ long long pv_slots(int d) { return kSms * (d == 64 ? 2 : 1); }
 void plan_rect(Plan &p, size_t budget) {
     const long long nRT = (p.L + 127) / 128;
     const size_t tile_bytes = size_t(128) * p.row_bytes;  // one 128-row tile of one head
-    const size_t head_bytes = size_t(p.L) * p.row_bytes;
+    const size_t head_bytes = size_t(nRT) * tile_bytes;   // the slab stores whole 128-row tiles
     const long long fit_tiles = static_cast<long long>(budget / tile_bytes);
     const long long fit_heads = static_cast<long long>(budget / head_bytes);
     long long best_cost = -1, best_groups = 0, best_nh = 1, best_rt = 1;
@@ -156,7 +156,9 @@ void plan_rect(Plan &p, size_t budget) {
     p.whole = p.R == p.L;
     p.gt = (p.L + p.R - 1) / p.R;
     p.ngroups = ((p.BH + p.Gh - 1) / p.Gh) * p.gt;
-    p.slab_bytes = align_up(size_t(p.Gh) * p.R * p.row_bytes, kAlign);
+    // whole 128-row tiles: the scores (4 Lp bytes a row) first, then the partials
+    const size_t rows = size_t(p.Gh) * ((p.R + 127) / 128) * 128;
+    p.slab_bytes = align_up(rows * p.Lp * 4, kAlign) + align_up(rows * (p.row_bytes - p.Lp * 4), kAlign);
     p.off_D = p.slab_bytes;
     p.total = p.off_D;
 }
@@ -383,6 +385,28 @@ bool map3d(CUtensorMap *m, CUtensorMapDataType type, const void *base, uint64_t 
                  static_cast<int>(r), base, static_cast<unsigned long long>(d0),
                  static_cast<unsigned long long>(d1), static_cast<unsigned long long>(d2), box0,
                  box1);
+        return false;
+    }
+    return true;
+}
+
+// The fp32 score slab of `tiles` (head, 128-row tile) units whose key chunks of 32 are
+// contiguous [128 rows][32 keys] blocks, `chunks` of them per unit and `unit_chunks` between
+// units: a 4-D tensor (32 keys, 128 rows, chunks, tiles), 128-byte swizzle, box (32, box_rows).
+bool map_slab(CUtensorMap *m, void *base, uint64_t chunks, uint64_t unit_chunks, uint64_t tiles,
+              uint32_t box_rows) {
+    cuuint64_t dims[4] = {32, 128, chunks, tiles};
+    cuuint64_t strides[3] = {128, 16384, unit_chunks * 16384};
+    cuuint32_t box[4] = {32, box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_err, sizeof(g_err),
+                 "cuTensorMapEncodeTiled failed (%d): slab base %p chunks %llu of %llu tiles %llu",
+                 static_cast<int>(r), base, static_cast<unsigned long long>(chunks),
+                 static_cast<unsigned long long>(unit_chunks), static_cast<unsigned long long>(tiles));
         return false;
     }
     return true;
@@ -687,16 +711,15 @@ rsa_status_t rsa_forward(const void *Q, const void *K, const void *V, void *O, f
     for (long long g = 0; g < p.ngroups; ++g) {
         const Group G = group_of(p, g);
         SlabArgs a = slab_args(p, G, dev->status);
-        const uint64_t pitch = uint64_t(p.Lp) * 4;  // fp32 row of the slab
+        // the slab: per (head, 128-row tile) unit, Lp / 32 contiguous [128 rows][32 keys] blocks
+        const uint64_t chunks = uint64_t(p.Lp) / 32, tiles = uint64_t(G.nh) * a.nRT;
         a.nCT = (p.Lp + 255) / 256;
         a.nStat = 2 * a.nCT;
         a.stats = reinterpret_cast<float2 *>(reinterpret_cast<uint8_t *>(slab) +
-                                             align_up(size_t(G.nh) * G.R * pitch, kAlign));
+                                             align_up(tiles * chunks * 16384, kAlign));
         CUtensorMap mS, mSld;
-        if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
-                   pitch * G.R, 32, 32) ||
-            !map3d(&mSld, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, slab, p.Lp, G.R, G.nh, pitch,
-                   pitch * G.R, 32, 128))
+        if (!map_slab(&mS, slab, chunks, chunks, tiles, 32) ||
+            !map_slab(&mSld, slab, chunks, chunks, tiles, 128))
             return RSA_ERR_CUDA;
         // ring pass 1: score slab and per-row softmax partials
         a.ntiles = G.nh * a.nRT * a.nCT;
@@ -843,13 +866,13 @@ rsa_status_t rsa_sp_scores(const void *Q, const void *Kfull, int B, int H, int L
     a.kcol0 = m * y.c, a.kend = (m + 1) * y.c, a.stat0 = m * 2 * y.nCT;
     a.stats = reinterpret_cast<float2 *>(ws + y.slab_bytes);
     a.ntiles = a.nh * a.nRT * a.nCT;
-    // the slab window of chunk m: columns [m c, (m + 1) c) of the rank's [BH][c][L] scores; the
-    // map's extent clips the stores of a tile that reaches past the window
-    const uint64_t pitch = uint64_t(y.Lp) * 4;
+    // the slab window of chunk m: key chunks [m c / 32, (m + 1) c / 32) of every (head, row
+    // tile) unit of the rank's scores; the map's extent clips the stores of a tile that reaches
+    // past the window
+    const uint64_t chunks = uint64_t(y.Lp) / 32, tiles = uint64_t(y.BH) * (y.c / 128);
     CUtensorMap mQ, mK, mS;
     if (!map_rows(&mQ, Q, y.BH, y.c, d, 128) || !map_rows(&mK, Kfull, y.BH, L, d, 256) ||
-        !map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws + size_t(m) * y.c * 4, y.c, y.c, y.BH,
-               pitch, pitch * y.c, 32, 32))
+        !map_slab(&mS, ws + size_t(m) * (y.c / 32) * 16384, y.c / 32, chunks, tiles, 32))
         return RSA_ERR_CUDA;
     RSA_LAUNCH(K_QK_SLAB, rsa::launch_qk_slab(mQ, mK, mS, a, dev->sms, s));
     return RSA_OK;
@@ -873,11 +896,10 @@ rsa_status_t rsa_sp_softmax_pv(const void *Vfull, void *O, float *lse, int B, in
     SlabArgs a = sp_slab_args(y, L, d, P, rank, causal, dev->status);
     a.stats = reinterpret_cast<float2 *>(ws + y.slab_bytes);
     a.ntiles = a.nh * a.nRT;
-    const uint64_t pitch = uint64_t(y.Lp) * 4;
+    const uint64_t chunks = uint64_t(y.Lp) / 32, tiles = uint64_t(y.BH) * (y.c / 128);
     CUtensorMap mS, mV, mO;
-    if (!map3d(&mS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws, y.Lp, y.c, y.BH, pitch, pitch * y.c, 32,
-               128) ||
-        !map_rows(&mV, Vfull, y.BH, L, d, 64) || !map_rows_out(&mO, O, y.BH, y.c, d))
+    if (!map_slab(&mS, ws, chunks, chunks, tiles, 128) || !map_rows(&mV, Vfull, y.BH, L, d, 64) ||
+        !map_rows_out(&mO, O, y.BH, y.c, d))
         return RSA_ERR_CUDA;
     RSA_LAUNCH(K_PV, rsa::launch_pv_softmax(mS, mV, mO, lse, a, dev->sms, s));
     return RSA_OK;
