@@ -9,6 +9,7 @@ in groups that fit the workspace budget. Prints one JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long|gpt|bert|f32|sweep]
     python bench.py --impl reference ...   # the fp64 CPU oracle on the same workload
+    python bench.py --ring P ...           # the ring across P GPUs, emulated on one GPU
 
 Timing: W untimed steps; then K steps, each preceded (outside the timed events) by an L2
 flush (a 512 MiB write) and a short GPU spin that keeps the launch queue ahead of the GPU;
@@ -693,6 +694,83 @@ def run_sweep(args):
     return 0
 
 
+def run_ring(args, w):
+    """The ring across GPUs, emulated on one GPU: every rank's per-rank kernels (rsa_sp_*, the
+    library's sequence-parallel steps) run in lockstep on this device and the exchange between
+    neighbours is a device copy (no kernel waits for another rank's). One JSON line with the
+    emulated step's time (all P ranks' work, the same 12pd flops as the single-device step),
+    the per-rank share, each kernel's roofline fraction, and the bytes per rank that NCCL would
+    move between GPUs (not timed here: every GPU run available has one GPU). Not the contract
+    line: an extra measurement of the ring's kernels."""
+    import torch
+
+    from sequence_ring_self_b200 import build, ring, rsa
+    from sequence_ring_self_b200.inputs import make_inputs
+
+    build.build()
+    rsa.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    P = args.ring
+    B, H, L, d, causal = w["B"], w["H"], w["L"], w["d"], w["causal"]
+    if L % P or (L // P) % 128:
+        raise SystemExit(f"the ring needs L / P to be a multiple of 128 (L={L}, P={P})")
+    c = L // P
+    x = make_inputs(B, H, L, d, seed=w["seed"], dtype="bf16")
+    q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+    comp = ring.Kernels()
+    chunk = lambda t, r: t[:, :, r * c:(r + 1) * c].contiguous()
+    states = [ring.RankState(q=chunk(q, r), kfull=ring.full_buffer(chunk(k, r), r, P),
+                             vfull=ring.full_buffer(chunk(v, r), r, P), causal=causal, do=chunk(do, r))
+              for r in range(P)]
+
+    def step():
+        rings = []
+        rings.extend(ring.LocalRing(r, states, rings) for r in range(P))
+        ring.run_lockstep([ring.forward_steps(states[r], rings[r], comp) for r in range(P)])
+        ring.run_lockstep([ring.backward_steps(states[r], rings[r], comp) for r in range(P)])
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    host_s = warm_up(step, max(3, args.warmup), flush)
+    guard = int(min(8e6, max(2e5, 4.0 * host_s * 2.0e9)))
+    times = timed_steps(step, args.steps, flush, guard, False)
+    kp = max(3, min(args.steps, args.profile_steps))
+    timed_steps(step, kp, flush, guard, True)
+    prof = rsa.profile_read()
+    rsa.profile_enable(False)
+    if rsa.last_device_status() != rsa.RSA_OK:
+        raise RuntimeError("a kernel reported a timeout")
+    ms = sum(times) / len(times)
+    peaks = load_peaks()
+    phases = phases_from_profile({n: v for n, v in prof.items() if n != "sp_accumulate"}, kp, w, peaks,
+                                 compute_peaks(peaks, {"reasons": []}, measure_ffma(dev)))
+    acc = prof.get("sp_accumulate")
+    acc_ms = acc[0] / kp if acc else 0.0
+    kernel_ms = sum(ph["ms_per_step"] for ph in phases) + acc_ms
+    chunk_bf16 = B * H * c * d * 2
+    line = {
+        "ring_emulated": {"ranks": P, "chunk_rows": c}, "workload": w["name"],
+        # the device time of every rank's kernels in one step (CUDA events per kernel): one
+        # GPU of a real P-GPU ring runs a P-th of it
+        "kernel_ms_per_step_all_ranks": kernel_ms, "kernel_ms_per_rank": kernel_ms / P,
+        "kernel_tflops_one_gpu": step_flops(w) / kernel_ms / 1e9,
+        # wall time of the emulated step on one GPU: host-bound when the per-rank problems are
+        # small (P * P steps of launches from one Python thread)
+        "wall_ms_per_step_all_ranks": ms,
+        "nccl_bytes_per_rank_step": {"forward_kv_chunks": 2 * (P - 1) * chunk_bf16,
+                                     "backward_dkdv_fp32_accumulators": 2 * (P - 1) * 2 * chunk_bf16},
+        "exchange": "device copies on one GPU (NCCL send/recv between GPUs: not measured here)",
+        "kernels": {ph["kernel"]: {"ms_per_step": ph["ms_per_step"], "launches_per_step": ph["launches_per_step"],
+                                   "bound": ph.get("bound"),
+                                   "frac": ph["hbm_frac"] if ph.get("bound") == "hbm" else ph.get("compute_frac")}
+                    for ph in phases},
+        "sp_accumulate_ms_per_step": acc_ms,
+        "roofline_e2e_of_kernel_time": roofline_e2e(phases, kernel_ms)["frac"],
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -718,6 +796,8 @@ def main():
     ap.add_argument("--profile-steps", type=int, default=10,
                     help="steps of the per-kernel profiled pass that follows the timed region")
     ap.add_argument("--flush-mib", type=int, default=512, help="L2 flush buffer (MiB) written before each step")
+    ap.add_argument("--ring", type=int, default=0,
+                    help="emulate the ring across this many GPUs on one GPU (extra line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -726,6 +806,8 @@ def main():
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.ring:
+        return run_ring(args, w)
     if args.forward == "recompute" and w["dtype"] != "bf16":
         ap.error("--forward recompute is bf16 only")
     return run_gpu(args, w)
