@@ -796,6 +796,8 @@ def main():
     ap.add_argument("--profile-steps", type=int, default=10,
                     help="steps of the per-kernel profiled pass that follows the timed region")
     ap.add_argument("--flush-mib", type=int, default=512, help="L2 flush buffer (MiB) written before each step")
+    ap.add_argument("--shape", default=None,
+                    help="B,H,L,d,N,causal: a bf16 workload of this shape instead of --workload")
     ap.add_argument("--ring", type=int, default=0,
                     help="emulate the ring across this many GPUs on one GPU (extra line)")
     args = ap.parse_args()
@@ -804,6 +806,11 @@ def main():
     if args.workload == "sweep":
         return run_sweep(args)
     w = WORKLOADS[args.workload]
+    if args.shape:
+        B, H, L, d, N, causal = (int(x) for x in args.shape.split(","))
+        w = dict(B=B, H=H, L=L, d=d, N=N, causal=bool(causal), seed=4, dtype="bf16",
+                 name=f"RSA fwd+bwd: B={B} H={H} L={L} d={d} N={N} bf16 "
+                      f"{'causal' if causal else 'non-causal'}")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.ring:
