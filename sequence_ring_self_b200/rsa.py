@@ -315,27 +315,107 @@ class RingSelfAttention(torch.autograd.Function):
         return dq, dk, dv, None, None
 
 
+def host_chunks(B: int, H: int, L: int, d: int, elsize: int = 2) -> int:
+    """How many groups of (batch, head) slices ``forward_backward_host`` pipelines: the most,
+    up to 8, that divides B H and still gives each group at least 8 MB of Q, K, V and dO to
+    copy. Issuing a group costs the host about a quarter of a millisecond, about what 8 MB
+    takes over PCIe, so smaller groups would leave the GPU waiting for the host."""
+    BH = B * H
+    for c in range(min(8, BH), 1, -1):
+        if BH % c == 0 and 4 * (BH // c) * L * d * elsize >= 8e6:
+            return c
+    return 1
+
+
 def forward_backward_host(q, k, v, do, N: int, causal: bool = False, *, ws_budget: int = 0,
-                          device=None, results=None, recompute: bool = False):
+                          device=None, results=None, recompute: bool = False,
+                          chunks: int | None = None):
     """One forward + backward from host (ideally pinned) tensors: copies Q, K, V, dO to the
     device, runs the library's forward and backward there, and copies O, lse, dQ, dK, dV
     back into host tensors (``results`` if given, a dict of pinned tensors by name).
-    ``recompute`` selects the slab-free forward."""
+    ``recompute`` selects the slab-free forward.
+
+    Attention is independent across the B H (batch, head) slices, so the call runs as a
+    pipeline over ``chunks`` groups of slices (default ``host_chunks``): the copies of group
+    c + 1 to the device (one side stream) overlap the forward of group c, dO arrives while the
+    forwards run, and O, lse and the gradients of each group go back to the host (a second
+    side stream, the other PCIe direction) while the next group computes. Every group is one
+    library call on [1, B H / chunks, L, d] views, so the results equal those of a single call
+    bit for bit. All work is ordered before the current stream's later work: synchronising the
+    current stream covers the results."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in (q, k, v, do))
-    if recompute:
-        o, lse = forward_recompute(qd, kd, vd, N, causal)
-    else:
-        o, lse = forward(qd, kd, vd, N, causal, ws_budget=ws_budget)
-    dq, dk, dv = backward(qd, kd, vd, o, dod, lse, N, causal, ws_budget=ws_budget)
-    names = ("O", "lse", "dQ", "dK", "dV")
-    if results is None:
-        results = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                   for n, t in zip(names, (o, lse, dq, dk, dv))}
-    for n, t in zip(names, (o, lse, dq, dk, dv)):
-        results[n].copy_(t, non_blocking=True)
+    B, H, L, d = q.shape
+    BH = B * H
+    C = host_chunks(B, H, L, d, q.element_size()) if chunks is None else int(chunks)
+    if C < 1 or BH % C:
+        raise ValueError(f"chunks = {C} must divide B H = {BH}")
+    n = BH // C
+    flat = lambda t: t.reshape(BH, *t.shape[2:])
+    piece = lambda t, c: flat(t)[c * n:(c + 1) * n]
+    with torch.cuda.device(dev):
+        main = torch.cuda.current_stream(dev)
+        h2d, d2h = _side_streams(dev)
+        if results is None:
+            results = {nm: torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+                       for nm in ("O", "dQ", "dK", "dV")}
+            results["lse"] = torch.empty((B, H, L), dtype=torch.float32, pin_memory=True)
+        # device buffers belong to the current stream; the side streams finish with them
+        # before it goes on (it waits on their events below and on d2h at the end)
+        qd, kd, vd, dod, o, dq, dk, dv = (torch.empty(q.shape, dtype=q.dtype, device=dev)
+                                          for _ in range(8))
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        h2d.wait_stream(main)  # host and device buffers may still be in use by earlier work
+        d2h.wait_stream(main)
+        in_ready, do_ready = [], []
+        with torch.cuda.stream(h2d):
+            for c in range(C):
+                for src, dst in ((q, qd), (k, kd), (v, vd)):
+                    piece(dst, c).copy_(piece(src, c), non_blocking=True)
+                in_ready.append(torch.cuda.Event())
+                in_ready[-1].record(h2d)
+            for c in range(C):
+                piece(dod, c).copy_(piece(do, c), non_blocking=True)
+                do_ready.append(torch.cuda.Event())
+                do_ready[-1].record(h2d)
+        view = lambda t, c: piece(t, c).unsqueeze(0)  # [1, n, L, d] or [1, n, L]
+        for c in range(C):
+            main.wait_event(in_ready[c])
+            if recompute:
+                forward_recompute(view(qd, c), view(kd, c), view(vd, c), N, causal,
+                                  out=view(o, c), lse=view(lse, c))
+            else:
+                forward(view(qd, c), view(kd, c), view(vd, c), N, causal, ws_budget=ws_budget,
+                        out=view(o, c), lse=view(lse, c))
+            done = torch.cuda.Event()
+            done.record(main)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                piece(results["O"], c).copy_(piece(o, c), non_blocking=True)
+                piece(results["lse"], c).copy_(piece(lse, c), non_blocking=True)
+        for c in range(C):
+            main.wait_event(do_ready[c])
+            backward(view(qd, c), view(kd, c), view(vd, c), view(o, c), view(dod, c),
+                     view(lse, c), N, causal, ws_budget=ws_budget, dq=view(dq, c),
+                     dk=view(dk, c), dv=view(dv, c))
+            done = torch.cuda.Event()
+            done.record(main)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                for nm, t in (("dQ", dq), ("dK", dk), ("dV", dv)):
+                    piece(results[nm], c).copy_(piece(t, c), non_blocking=True)
+        main.wait_stream(d2h)
     return results
 
+
+_SIDE = {}
+
+
+def _side_streams(dev):
+    """Two side streams per device (host-to-device and device-to-host copies), made once."""
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _SIDE:
+        _SIDE[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _SIDE[key]
 
 def linear(x, w, bias=None, residual=None, gelu: bool = False, *, x_kin: int | None = None,
            y_kin: int | None = None, out=None, stream: torch.cuda.Stream | None = None):

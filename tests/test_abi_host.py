@@ -220,3 +220,20 @@ def test_linear_argument_errors(lib):
     assert _lin(lib, K=96, xk=96) == rsa.RSA_ERR_UNSUPPORTED      # K not a multiple of 64
     assert _lin(lib, K=256, xk=96) == rsa.RSA_ERR_UNSUPPORTED     # head width not dividing K
     assert _lin(lib, N=128, yk=64, res=FAKE) == rsa.RSA_ERR_UNSUPPORTED  # residual, split output
+
+
+def test_host_pipeline_chunking_rule():
+    """Groups of (batch, head) slices for the host-buffer call: at most 8, dividing B H, each
+    with at least 8 MB of Q, K, V, dO (the choices measured fastest on the long-sequence,
+    GPT-style and BERT-shaped steps: 8, 8 and 3)."""
+    from sequence_ring_self_b200.rsa import host_chunks
+
+    assert host_chunks(1, 16, 16384, 128) == 8
+    assert host_chunks(4, 16, 4096, 64) == 8
+    assert host_chunks(8, 12, 512, 64) == 3
+    assert host_chunks(1, 2, 256, 64) == 1
+    assert host_chunks(1, 7, 65536, 128) == 7
+    for B, H, L, d, e in ((1, 16, 16384, 128, 2), (2, 5, 9000, 64, 4), (3, 5, 7000, 64, 2)):
+        c = host_chunks(B, H, L, d, e)
+        assert 1 <= c <= 8 and (B * H) % c == 0
+        assert c == 1 or 4 * (B * H // c) * L * d * e >= 8e6

@@ -320,6 +320,33 @@ def test_autograd_wrapper_and_host_api(orc):
         np.testing.assert_array_equal(res[n].to(torch.float64).numpy(), ref[n])
 
 
+@pytest.mark.parametrize("shape,chunks", [((2, 3, 384, 64, 3, True), 2),
+                                          ((2, 3, 384, 64, 3, True), 6),
+                                          ((1, 4, 300, 128, 3, False), 4)])
+@pytest.mark.parametrize("recompute", [False, True])
+def test_host_api_pipeline_equals_one_call(orc, shape, chunks, recompute):
+    """The host-buffer call cut into groups of (batch, head) slices gives the single call's
+    results bit for bit, and those agree with the oracle."""
+    B, H, L, d, N, causal = shape
+    x = make_inputs(B, H, L, d, seed=9 + chunks, dtype="bf16")
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (x.torch(n, dev) for n in ("q", "k", "v", "do"))
+    if recompute:
+        o, lse = rsa.forward_recompute(q, k, v, N, causal)
+    else:
+        o, lse = rsa.forward(q, k, v, N, causal)
+    dq, dk, dv = rsa.backward(q, k, v, o, do, lse, N, causal)
+    one = {"O": o, "lse": lse, "dQ": dq, "dK": dk, "dV": dv}
+    host = {n: x.torch(n).pin_memory() for n in ("q", "k", "v", "do")}
+    res = rsa.forward_backward_host(host["q"], host["k"], host["v"], host["do"], N, causal,
+                                    chunks=chunks, recompute=recompute)
+    torch.cuda.synchronize()
+    assert rsa.last_device_status() == rsa.RSA_OK
+    for n in one:
+        np.testing.assert_array_equal(res[n].to(torch.float64).numpy(), np64(one[n]), err_msg=n)
+    check_full(orc, x, {n: res[n].to(torch.float64).numpy() for n in one}, causal)
+
+
 RECOMPUTE_SHAPES = [  # (B, H, L, d, N, causal)
     (2, 3, 512, 64, 4, False),
     (2, 3, 512, 64, 4, True),
