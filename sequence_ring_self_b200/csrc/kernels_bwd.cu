@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->sfull[b], 1);
-            mbar_init(&ctl->pready[b], kEpiWarps);
+            mbar_init(&ctl->pready[b], 1);  // one epilogue warp posts for all eight
         }
         mbar_init(&ctl->accfull, 1);
         mbar_init(&ctl->accempty, kEpiWarps);
@@ -412,7 +412,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         uint32_t gstep = 0, acc_ph = 0;
         Pipe ps{0, 0};  // the Q/dO stage of the current step (same order as the producer's)
         bool ok = true;
-        uint32_t total = 0;  // steps of this CTA (pready(g) vouches for stage g + 2)
+        bool vouched = true;  // epilogue warp 0: its last wait for a stage g + 2 succeeded
+        uint32_t total = 0;   // steps of this CTA (pready(g) vouches for stage g + 2)
         for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
             BkTile tl;
             if (bk_decode(a, t, tl)) total += tl.cnt;
@@ -427,8 +428,15 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 const int i0 = a.r0 + bk_block(tl, s) * 64;
                 const int ic = i0 + 32 * hf;  // first query column of this warp
                 const int r_end = a.r0 + a.R;
-                if (!warp_wait(&ctl->sfull[b], bph, &ctl->abort) ||
-                    !warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort)) {
+                // Epilogue warp 0 polls the barriers for all eight and the named barrier releases
+                // them together (with its verdict). The tensor core keeps the shared-memory
+                // port busy, so every poll waits for it: one poller instead of eight, and no
+                // warp that started waiting early and notices late.
+                bool good = vouched;
+                if (ew == 0 && good)
+                    good = warp_wait(&ctl->sfull[b], bph, &ctl->abort) &&
+                           warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort);
+                if (!group_all(good, kEpiWarps * 32)) {
                     ok = false;
                     break;
                 }
@@ -453,24 +461,28 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tmem_st16(t_s + 64, wd);
                 tmem_st_wait();
                 tc_fence_before();
-                if (gstep + 2 < total) {
-                    Pipe p2 = ps;
-                    pipe_next(p2, C::STAGES);
-                    pipe_next(p2, C::STAGES);
-                    if (!warp_wait(&ctl->full[p2.stage], p2.phase, &ctl->abort)) {
-                        ok = false;
-                        break;
+                group_sync(kEpiWarps * 32);  // every warp's P^T/dS^T is in TMEM
+                if (ew == 0) {
+                    if (gstep + 2 < total) {
+                        Pipe p2 = ps;
+                        pipe_next(p2, C::STAGES);
+                        pipe_next(p2, C::STAGES);
+                        vouched = warp_wait(&ctl->full[p2.stage], p2.phase, &ctl->abort);
                     }
+                    // a failed wait posts nothing: the next step's named barrier carries it
+                    if (vouched && lane == 0) mbar_arrive(&ctl->pready[b]);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->pready[b]);
                 ++gstep;
                 pipe_next(ps, C::STAGES);
             }
             if (!ok) break;
             // dV_m and dK_m of this key tile (scale dS^T Q for dK), bf16 through the staging
-            // buffer: warp (q, hf) stores keys j0 + 32q .. +31, columns hf*D/2 .. +D/2
-            if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
+            // buffer: warp (q, hf) stores keys j0 + 32q .. +31, columns hf*D/2 .. +D/2. The
+            // eight warps take every wait's verdict from the same poll, so none of them can
+            // leave the named-barrier sequence while another stays in it.
+            bool acc_ok = true;
+            if (ew == 0) acc_ok = warp_wait(&ctl->accfull, acc_ph, &ctl->abort);
+            if (!group_all(acc_ok, kEpiWarps * 32)) break;
             tc_fence_after();
             const int jw = tl.j0 + 32 * q;
 #pragma unroll 1

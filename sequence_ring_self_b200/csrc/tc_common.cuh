@@ -54,6 +54,27 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok != 0;
 }
 
+// Named barrier 1 over `nthreads` threads (whole warps): every participant waits for all,
+// and learns whether all passed `pred` (bar.red.and). It uses the SM's barrier unit, not
+// shared memory, so one warp can poll an mbarrier on behalf of a group of warps while the
+// tensor core keeps the shared-memory port busy.
+__device__ __forceinline__ bool group_all(bool pred, int nthreads) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void group_sync(int nthreads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void init_ctl(Ctl *ctl, int stages, int tempty_count) {
     for (int s = 0; s < stages; ++s) {
         mbar_init(&ctl->full[s], 1);
