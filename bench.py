@@ -624,6 +624,7 @@ def run_gpu(args, w):
                                    "workspace_bytes": [wl.nf, wl.nb]}},
         "tokens_per_s": tokens_s,
         "step_ms_median": statistics.median(step_ms),
+        "step_ms_min": min(step_ms),
         "e2e": e2e,
         "gpu_launches": int(round(sum(n for _, n in prof.values()) / kp * K)),
         "profiled_pass": {"steps": kp, "ms_per_step_with_kernel_events": statistics.median(prof_step_ms)},
@@ -785,7 +786,7 @@ def main():
     ap.add_argument("--sweep-N", default="1,2,4,8,16")
     ap.add_argument("--sweep-steps", type=int, default=5)
     ap.add_argument("--ws-budget", type=int, default=0, help="workspace budget in bytes (0: default)")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
                     help="CPU seconds of the oracle sample reported as cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds the whole --impl reference run should take")

@@ -237,3 +237,14 @@ def test_host_pipeline_chunking_rule():
         c = host_chunks(B, H, L, d, e)
         assert 1 <= c <= 8 and (B * H) % c == 0
         assert c == 1 or 4 * (B * H // c) * L * d * e >= 8e6
+
+
+@pytest.mark.parametrize("chunks", [0, 3, -2])
+def test_host_pipeline_rejects_groups_that_do_not_divide_the_slices(chunks):
+    """B H = 4 (batch, head) slices cannot be cut into 0, 3 or -2 groups; the call says so
+    before it touches a device."""
+    from sequence_ring_self_b200 import rsa
+
+    x = torch.zeros(2, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rsa.forward_backward_host(x, x, x, x, 4, False, device="cuda:0", chunks=chunks)

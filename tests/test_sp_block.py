@@ -1,5 +1,5 @@
-"""The Transformer block under sequence parallelism (the survey's "next" row for the block's
-linear layers): each rank's linear layers on its own rows, Ring Self-Attention across the ranks,
+"""The Transformer block under sequence parallelism (the block's linear layers around the
+attention): each rank's linear layers on its own rows, Ring Self-Attention across the ranks,
 against the fp64 oracle composed on the whole sequence (oracle.linear and oracle.forward).
 
 * CPU: real gloo processes (world 2, causal and not) run `block.block_forward` with fp64
