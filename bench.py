@@ -423,6 +423,58 @@ def measure_ffma(dev, reps: int = 5):
     return flops / (best / 1e3) / 1e12
 
 
+# the slab kernels' traffic is almost all one direction: scores written, or scores read
+SLAB_DIRECTION = {"qk_slab": "write", "pv_softmax": "read"}
+
+
+def measure_hbm(dev, reps: int = 5):
+    """HBM read-only and write-only streaming rates of this GPU (GB/s), from the library's probe
+    kernels over a buffer far above the L2 size, timed with CUDA events (best of `reps`)."""
+    import ctypes
+
+    import torch
+
+    from sequence_ring_self_b200 import rsa
+
+    lib = rsa.load_library()
+    free, _ = torch.cuda.mem_get_info(dev)
+    nbytes = min(2 << 30, (free // 4) // (1 << 20) * (1 << 20))
+    if nbytes < (512 << 20):
+        return None  # too little free memory for a buffer well above L2
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = sms * 8
+    out = torch.empty(blocks, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    rates = {}
+    for name, write in (("write", 1), ("read", 0)):
+        best = None
+        for _ in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            rc = lib.rsa_probe_hbm(ctypes.c_void_p(buf.data_ptr()), nbytes, write, blocks,
+                                   ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(s.cuda_stream))
+            e1.record(s)
+            if rc != rsa.RSA_OK:
+                raise rsa.RSAError(rc, "rsa_probe_hbm")
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        rates[name] = nbytes / (best / 1e3) / 1e9
+    del buf, out
+    return rates
+
+
+def annotate_directions(phases, hbm_probe):
+    """Each slab kernel's achieved GB/s against the probe rate of its traffic's direction."""
+    if not hbm_probe:
+        return
+    for ph in phases:
+        direction = SLAB_DIRECTION.get(ph["kernel"])
+        if direction and "achieved_gbs" in ph:
+            ph["hbm_frac_of_" + direction + "_probe"] = ph["achieved_gbs"] / hbm_probe[direction]
+
+
 class Workload:
     """Device tensors, workspaces and the step function of one workload on one GPU."""
 
@@ -592,8 +644,10 @@ def run_gpu(args, w):
 
     peaks = load_peaks()
     ffma = measure_ffma(dev)
+    hbm_probe = measure_hbm(dev)
     clock_rec = clocks.summary(t0, t1)
     phases = phases_from_profile(prof, kp, w, peaks, compute_peaks(peaks, clock_rec, ffma))
+    annotate_directions(phases, hbm_probe)
     if not phases:
         phases = [{"kernel": "none (no per-kernel events)"}]
     traffic = None
@@ -632,7 +686,9 @@ def run_gpu(args, w):
         "roofline_e2e": roofline_e2e(phases, step_ms_avg),
         "phases": phases,
         "clocks": clock_rec,
-        "peaks": dict(peaks, ffma_tflops_this_run=ffma),
+        "peaks": dict(peaks, ffma_tflops_this_run=ffma,
+                      hbm_read_gbs_this_run=hbm_probe and hbm_probe["read"],
+                      hbm_write_gbs_this_run=hbm_probe and hbm_probe["write"]),
     }
     if world == 1 and not args.no_cpu_baseline:
         fl, sec, desc, threads = oracle_sample(w, args.cpu_seconds)

@@ -191,6 +191,24 @@ RSA_API rsa_status_t rsa_profile_read(double *ms, long long *launches);
 RSA_API rsa_status_t rsa_probe_ffma(void *out, int blocks, int iters, void *stream);
 RSA_API long long rsa_probe_ffma_flops_per_thread(int iters);
 
+/*
+ * HBM streaming probe (a benchmark helper, not part of the method): context for the slab
+ * kernels, whose traffic is almost all writes (the scores) or almost all reads (softmax/PV).
+ * Launches `blocks` blocks of 256 threads on `stream` that read (write = 0) or write
+ * (write = 1) every byte of `buf` once, in 16-byte vectors, four independent ones per thread
+ * and iteration. The caller times the launch (CUDA events on `stream`) and divides `bytes` by
+ * the time; `bytes` should be far above the L2 size (126 MB) so that the rate is HBM's.
+ * buf: device buffer of `bytes` bytes, 16-byte aligned, bytes a positive multiple of 16; the
+ * write probe fills it with a pattern (word k of 16-byte vector i holds i + k, modulo 2^32).
+ * out: device buffer of at least `blocks` 32-bit words for the read probe (written only in a
+ * case that never occurs, so that the compiler keeps the loads); may be NULL for the write
+ * probe. Returns RSA_ERR_INVALID_ARG for a NULL or misaligned buffer, a size that is not a
+ * positive multiple of 16, non-positive blocks, write not 0 or 1, or a read probe without
+ * `out`; RSA_ERR_CUDA if the launch fails.
+ */
+RSA_API rsa_status_t rsa_probe_hbm(void *buf, size_t bytes, int write, int blocks, void *out,
+                                   void *stream);
+
 /* Size of the scratch array rsa_forward_noalloc works in: 32 MiB of device memory per GPU
  * that loads the library, held until the process exits. */
 #define RSA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

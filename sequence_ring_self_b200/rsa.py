@@ -28,7 +28,8 @@ EXPORTED = ("rsa_workspace_size", "rsa_forward", "rsa_backward", "rsa_status_str
             "rsa_last_device_status", "rsa_plan_describe", "rsa_profile_enable",
             "rsa_profile_kinds", "rsa_profile_kind_name", "rsa_profile_read",
             "rsa_forward_noalloc", "rsa_last_error", "rsa_forward_recompute",
-            "rsa_probe_ffma", "rsa_probe_ffma_flops_per_thread", "rsa_debug_report_status",
+            "rsa_probe_ffma", "rsa_probe_ffma_flops_per_thread", "rsa_probe_hbm",
+            "rsa_debug_report_status",
             # include/rsa_sp.h
             "rsa_sp_workspace_size", "rsa_sp_scores", "rsa_sp_softmax_pv", "rsa_sp_backward_rows",
             "rsa_sp_backward_keys", "rsa_sp_accumulate", "rsa_linear")
@@ -92,6 +93,8 @@ def load_library(path: str | None = None):
         lib.rsa_probe_ffma.restype = i
         lib.rsa_probe_ffma_flops_per_thread.argtypes = [i]
         lib.rsa_probe_ffma_flops_per_thread.restype = ctypes.c_longlong
+        lib.rsa_probe_hbm.argtypes = [vp, sz, i, i, vp, vp]
+        lib.rsa_probe_hbm.restype = i
         lib.rsa_debug_report_status.argtypes = [i, vp]
         lib.rsa_debug_report_status.restype = i
         lib.rsa_linear.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]

@@ -1,6 +1,7 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads, exports every function
 ``include/rsa.h`` declares, rejects bad arguments before launching anything, and plans its
 workspace consistently."""
+import ctypes
 import os
 import re
 
@@ -248,3 +249,17 @@ def test_host_pipeline_rejects_groups_that_do_not_divide_the_slices(chunks):
     x = torch.zeros(2, 2, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         rsa.forward_backward_host(x, x, x, x, 4, False, device="cuda:0", chunks=chunks)
+
+
+def test_hbm_probe_argument_errors(lib):
+    """The HBM probe refuses bad buffers, sizes, block counts and modes before any launch."""
+    vp = ctypes.c_void_p
+    probe = lambda buf=FAKE, n=1 << 20, write=0, blocks=8, out=FAKE: lib.rsa_probe_hbm(
+        vp(buf), n, write, blocks, vp(out), vp(0))
+    assert probe(buf=0) == rsa.RSA_ERR_INVALID_ARG
+    assert probe(buf=FAKE + 8) == rsa.RSA_ERR_INVALID_ARG       # not 16-byte aligned
+    assert probe(n=0) == rsa.RSA_ERR_INVALID_ARG
+    assert probe(n=(1 << 20) + 8) == rsa.RSA_ERR_INVALID_ARG    # not a multiple of 16
+    assert probe(blocks=0) == rsa.RSA_ERR_INVALID_ARG
+    assert probe(write=2) == rsa.RSA_ERR_INVALID_ARG
+    assert probe(out=0) == rsa.RSA_ERR_INVALID_ARG              # the read probe needs `out`

@@ -89,3 +89,19 @@ def test_row_sample_spreads_over_the_sequence():
     assert rows[0] == 0 and rows[-1] == 16383 and len(rows) == 5
     w = dict(L=8, d=2, causal=True)
     assert bench._row_flops(w, [0, 7]) == 8.0 * (1 + 8) * 2
+
+
+def test_slab_kernels_are_compared_with_their_direction():
+    """The score kernel (writes) against the write probe, softmax/PV (reads) against the read
+    probe; other kernels and a missing probe add nothing."""
+    b = _bench()
+    phases = [{"kernel": "qk_slab", "achieved_gbs": 5000.0},
+              {"kernel": "pv_softmax", "achieved_gbs": 4800.0},
+              {"kernel": "bwd_keys", "achieved_gbs": 500.0}]
+    b.annotate_directions(phases, {"read": 6000.0, "write": 6250.0})
+    assert phases[0]["hbm_frac_of_write_probe"] == pytest.approx(0.8)
+    assert phases[1]["hbm_frac_of_read_probe"] == pytest.approx(0.8)
+    assert not any(k.startswith("hbm_frac_of") for k in phases[2])
+    fresh = [{"kernel": "qk_slab", "achieved_gbs": 5000.0}]
+    b.annotate_directions(fresh, None)
+    assert list(fresh[0]) == ["kernel", "achieved_gbs"]

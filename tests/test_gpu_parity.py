@@ -433,3 +433,36 @@ def test_library_errors_raise():
     with pytest.raises(rsa.RSAError) as e:
         rsa.forward(q2, q2, q2, 1, workspace=small)
     assert e.value.code == rsa.RSA_ERR_WORKSPACE
+
+
+def test_hbm_probe_writes_its_pattern_and_streams():
+    """The HBM probe's write kernel covers every 16-byte vector with its documented pattern
+    (word k of vector i holds i + k), and both directions stream at a plausible HBM rate."""
+    dev = torch.device("cuda", 0)
+    lib = rsa.load_library()
+    nbytes, blocks = 512 << 20, 148 * 8
+    buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    out = torch.zeros(blocks, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    vp = ctypes.c_void_p
+    rates = {}
+    for write in (1, 0):
+        best = None
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            rc = lib.rsa_probe_hbm(vp(buf.data_ptr()), nbytes, write, blocks, vp(out.data_ptr()),
+                                   vp(s.cuda_stream))
+            e1.record(s)
+            assert rc == rsa.RSA_OK
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        rates[write] = nbytes / (best / 1e3) / 1e9
+    words = buf.view(torch.int32).view(-1, 4).cpu()
+    nvec = nbytes // 16
+    for i in (0, 1, 12345, nvec // 2 + 7, nvec - 1):
+        assert words[i].tolist() == [i, i + 1, i + 2, i + 3], i
+    assert int((words[:, 1] - words[:, 0] != 1).sum()) == 0
+    for write, gbs in rates.items():
+        assert 1000.0 < gbs < 20000.0, (write, gbs)
