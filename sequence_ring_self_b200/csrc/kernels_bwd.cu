@@ -502,8 +502,8 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ control warp
-        // Polls every barrier the epilogue warps wait on and releases them through named
-        // barrier 1 (bar.red.and carries its verdict), so none of them touches shared memory to
+        // Polls every barrier the epilogue warps wait on and releases them through a named
+        // barrier (bar.red.and carries its verdict), so none of them touches shared memory to
         // poll: the tensor core keeps the port busy, every poll waits for it, and a warp that
         // starts polling early notices late. While they compute a step it checks that the
         // Q/dO stage two steps ahead has landed (pready(g) vouches for it); once their P^T/dS^T
