@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             const int bh = a.bh0 + tl.h;
             const int j = tl.j0 + 32 * q + lane;  // this thread's key
             for (int s = 0; s < tl.cnt; ++s) {
-                const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
+                const uint32_t b = gstep & 1u;
                 const int i0 = a.r0 + bk_block(tl, s) * 64;
                 const int ic = i0 + 32 * hf;  // first query column of this warp
                 const int r_end = a.r0 + a.R;
