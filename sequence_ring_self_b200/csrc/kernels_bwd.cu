@@ -33,10 +33,8 @@ namespace {
 
 using namespace tc;
 
+constexpr int kBkThreads = 320;
 constexpr int kEpiWarps = 8;
-// key-major kernel: producer, MMA issuer, eight epilogue warps and a control warp
-constexpr int kBkThreads = 32 * (3 + kEpiWarps);
-constexpr int kBkGroup = 32 * (kEpiWarps + 1);  // the epilogue warps and the control warp
 
 template <int D>
 struct BkCfg {
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(kBkThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->sfull[b], 1);
-            mbar_init(&ctl->pready[b], 1);  // one epilogue warp posts for all eight
+            mbar_init(&ctl->pready[b], kEpiWarps);
         }
         mbar_init(&ctl->accfull, 1);
         mbar_init(&ctl->accempty, kEpiWarps);
@@ -404,28 +402,33 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             drain_wait(&ctl->drain, 0);
         }
         __syncwarp();
-    } else if (warp < 2 + kEpiWarps) {
+    } else {
         // ------------------------------------------------------------------ epilogue
         const int ew = warp - 2, q = warp & 3, hf = ew >> 2;
         const float sl2 = a.scale * kLog2e;
         const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
         uint8_t *obase = smem + C::OFF_OUT + ew * C::OUT_BUFS * 2048;
         int obuf = 0;
-        uint32_t gstep = 0;
+        uint32_t gstep = 0, acc_ph = 0;
         Pipe ps{0, 0};  // the Q/dO stage of the current step (same order as the producer's)
         bool ok = true;
+        uint32_t total = 0;  // steps of this CTA (pready(g) vouches for stage g + 2)
+        for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+            BkTile tl;
+            if (bk_decode(a, t, tl)) total += tl.cnt;
+        }
         for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
             BkTile tl;
             if (!bk_decode(a, t, tl)) continue;
             const int bh = a.bh0 + tl.h;
             const int j = tl.j0 + 32 * q + lane;  // this thread's key
             for (int s = 0; s < tl.cnt; ++s) {
-                const uint32_t b = gstep & 1u;
+                const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
                 const int i0 = a.r0 + bk_block(tl, s) * 64;
                 const int ic = i0 + 32 * hf;  // first query column of this warp
                 const int r_end = a.r0 + a.R;
-                // released by the control warp once S^T/dP^T and the stage are ready (its verdict)
-                if (!group_all(true, kBkGroup)) {
+                if (!warp_wait(&ctl->sfull[b], bph, &ctl->abort) ||
+                    !warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort)) {
                     ok = false;
                     break;
                 }
@@ -450,16 +453,24 @@ __global__ void __launch_bounds__(kBkThreads, 1)
                 tmem_st16(t_s + 64, wd);
                 tmem_st_wait();
                 tc_fence_before();
-                group_sync(kBkGroup);  // every warp's P^T/dS^T is in TMEM: the control warp posts it
+                if (gstep + 2 < total) {
+                    Pipe p2 = ps;
+                    pipe_next(p2, C::STAGES);
+                    pipe_next(p2, C::STAGES);
+                    if (!warp_wait(&ctl->full[p2.stage], p2.phase, &ctl->abort)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->pready[b]);
                 ++gstep;
                 pipe_next(ps, C::STAGES);
             }
             if (!ok) break;
             // dV_m and dK_m of this key tile (scale dS^T Q for dK), bf16 through the staging
-            // buffer: warp (q, hf) stores keys j0 + 32q .. +31, columns hf*D/2 .. +D/2. The
-            // eight warps take every wait's verdict from the same poll, so none of them can
-            // leave the named-barrier sequence while another stays in it.
-            if (!group_all(true, kBkGroup)) break;  // the control warp saw the accumulators done
+            // buffer: warp (q, hf) stores keys j0 + 32q .. +31, columns hf*D/2 .. +D/2
+            if (!warp_wait(&ctl->accfull, acc_ph, &ctl->abort)) break;
             tc_fence_after();
             const int jw = tl.j0 + 32 * q;
 #pragma unroll 1
@@ -497,54 +508,10 @@ __global__ void __launch_bounds__(kBkThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->accempty);
+            acc_ph ^= 1u;
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------------ control warp
-        // Polls every barrier the epilogue warps wait on and releases them through a named
-        // barrier (bar.red.and carries its verdict), so none of them touches shared memory to
-        // poll: the tensor core keeps the port busy, every poll waits for it, and a warp that
-        // starts polling early notices late. While they compute a step it checks that the
-        // Q/dO stage two steps ahead has landed (pready(g) vouches for it); once their P^T/dS^T
-        // stores are done it posts pready. Every named-barrier operation is executed by all
-        // nine warps in the same order, and the only exits follow a shared verdict.
-        uint32_t gstep = 0, acc_ph = 0;
-        Pipe ps{0, 0};
-        bool ok = true, vouched = true;
-        uint32_t total = 0;  // steps of this CTA
-        for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
-            BkTile tl;
-            if (bk_decode(a, t, tl)) total += tl.cnt;
-        }
-        for (int t = blockIdx.x; ok && t < a.ntiles; t += gridDim.x) {
-            BkTile tl;
-            if (!bk_decode(a, t, tl)) continue;
-            for (int s = 0; s < tl.cnt; ++s) {
-                const uint32_t b = gstep & 1u, bph = (gstep >> 1) & 1u;
-                const bool good = vouched && warp_wait(&ctl->sfull[b], bph, &ctl->abort) &&
-                                  warp_wait(&ctl->full[ps.stage], ps.phase, &ctl->abort);
-                if (!group_all(good, kBkGroup)) {
-                    ok = false;
-                    break;
-                }
-                if (gstep + 2 < total) {
-                    Pipe p2 = ps;
-                    pipe_next(p2, C::STAGES);
-                    pipe_next(p2, C::STAGES);
-                    vouched = warp_wait(&ctl->full[p2.stage], p2.phase, &ctl->abort);
-                }
-                group_sync(kBkGroup);
-                // a failed wait posts nothing: the next named barrier carries it
-                if (vouched && lane == 0) mbar_arrive(&ctl->pready[b]);
-                ++gstep;
-                pipe_next(ps, C::STAGES);
-            }
-            if (!ok) break;
-            const bool acc_ok = vouched && warp_wait(&ctl->accfull, acc_ph, &ctl->abort);
-            if (!group_all(acc_ok, kBkGroup)) break;
-            acc_ph ^= 1u;
-        }
     }
 
     tc_fence_before();

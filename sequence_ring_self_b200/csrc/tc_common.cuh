@@ -54,35 +54,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok != 0;
 }
 
-// Named barriers over a group of `nthreads` threads (whole warps). They use the SM's barrier
-// unit, not shared memory, so one warp can poll an mbarrier on behalf of a group of warps while
-// the tensor core keeps the shared-memory port busy. A barrier must not serve both a reduction
-// (bar.red) and a plain sync (bar.sync): PTX leaves that mix undefined, so group_all uses
-// barrier 1 and group_sync barrier 2, each always with the same group. Both are the .aligned
-// forms, which count a warp correctly only if it arrives converged, so each first reconverges
-// the warp (code before them may have branched on the lane).
-//
-// group_all: every participant waits for all and learns whether all passed `pred`.
-__device__ __forceinline__ bool group_all(bool pred, int nthreads) {
-    uint32_t r;
-    __syncwarp();
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, %2, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(pred ? 1u : 0u), "r"(nthreads)
-        : "memory");
-    return r != 0;
-}
-
-// group_sync: every participant waits for all.
-__device__ __forceinline__ void group_sync(int nthreads) {
-    __syncwarp();
-    asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
-}
-
 __device__ __forceinline__ void init_ctl(Ctl *ctl, int stages, int tempty_count) {
     for (int s = 0; s < stages; ++s) {
         mbar_init(&ctl->full[s], 1);
